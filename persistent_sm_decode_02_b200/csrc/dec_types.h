@@ -1,0 +1,150 @@
+// Plan structures shared by the host planner and the device engine.
+//
+// One decode step is a static list of ops in topological order; every op is
+// cut into independent tile tasks.  The persistent kernel gives each CTA a
+// fixed list of (op, task) pairs; a task of op k waits until the counters of
+// k's dependencies reach epoch * ntasks, runs, and adds 1 to k's counter.  The
+// tile-level task decomposition with overlapped weight streaming is the
+// mechanism the pages describe for TileRT's engine ("Tile A1 + Tile B1 +
+// comm C1", TileRT 是什么 §二 2.2; InferenceX article, "what TileRT is").
+#pragma once
+#include <stdint.h>
+
+namespace dec {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;  // threads that compute
+constexpr int kThreads = kConsumers + 32;        // + one producer warp that streams weights
+constexpr int kStageBytes = 32768;               // one ring stage
+constexpr int kStages = 5;                       // ring depth (160 KB in flight per SM)
+constexpr int kWorkBytes = 48 * 1024;            // per-task scratch (input vector / attention state)
+constexpr int kMaxSegs = 20;
+constexpr int kMaxTopK = 16;
+constexpr int kMaxD = 8192;                      // longest normalised vector (d_model, q_lora)
+constexpr int kMlaHeadsPerTask = 16;             // heads per CUDA-core MLA attention task
+
+enum WType : int { WT_F32 = 0, WT_BF16 = 1, WT_FP8 = 2 };
+enum OpKind : int { OP_GEMV = 0, OP_ATTN = 1, OP_MLA = 2, OP_FINAL = 3 };
+enum Pro : int {
+  PRO_NONE = 0,
+  PRO_RESID_NORM = 1,   // h = base + partial sums (+ routed experts); x = R(rmsnorm(h) * g)
+  PRO_NORM_SUM = 2,     // x = R(rmsnorm(sum of partials) * g)
+  PRO_SUM = 3,          // x = R(sum of partials) (optionally per input group)
+  PRO_SWIGLU = 4,       // x = R(silu(gate) * up)
+  PRO_ATTN_COMBINE = 5, // x = R(split-KV log-sum-exp combine) for all heads
+  PRO_MLA_COMBINE = 6   // x = R(split-KV combine of one head's latent output)
+};
+
+// value(e) = sum_{s < S} ptr[s * stride + off + e]
+struct PSet {
+  const float* ptr;
+  int S, stride, off;
+};
+
+struct Seg {
+  const uint8_t* w;   // tiled weights (expert 0 for routed segments)
+  const float* sc;    // fp8 block scales [ceil(N/128)][ceil(K/128)] (expert 0 for routed segments)
+  long long w_estride;  // bytes between experts
+  long long s_estride;  // floats between experts' scale tables
+  int slot;           // routed slot j: weights of the router's j-th expert; -1: fixed weights
+  int N;              // rows
+  int ntiles;         // row tiles of R rows
+  int task0;          // first task of this segment within the op
+  int out_off;        // element offset of row 0 in every split's output
+  int in_group;       // prologue input variant shared by all tasks of the segment (-1: by row group)
+};
+
+struct OpDesc {
+  int kind, ntasks, layer;
+  int dep[2];  // consumer dependencies (op index or -1)
+  int pdep;    // producer dependency: router op whose top-k picks the weights of routed segments
+  // ---- GEMV geometry: a task = R rows x (nst stages of kc columns)
+  int wtype, K, Kpad, kcb, kc, cpr, G, rpt, R, S, nst;
+  int nsegs;
+  Seg seg[kMaxSegs];
+  int rows_per_group;  // grouped GEMV: input group = row / rows_per_group (0: one input for all rows)
+  float* out;          // fp32 partial outputs [S][out_stride]
+  int out_stride;
+  unsigned long long* best;  // LM head: best packed (value, index) key per task, else null
+  // ---- prologue
+  int pro;
+  int in_bf16;  // input vector dtype: 1 = bf16 (rounded), 0 = fp32
+  int n;        // input vector length (<= Kpad)
+  int base_embed;  // RESID_NORM: 1 = base is the embedding row of the step token
+  const void* embed;
+  int embed_bf16;
+  const float* h_base;
+  PSet add, add2;          // summed with weight 1 (ptr null = unused)
+  PSet routed;             // routed expert outputs, slot j at off + j * routed_slot_stride
+  int routed_slot_stride;
+  PSet route_logits;       // router logits (E values)
+  int n_experts, top_k;
+  int* route_dump;         // routed GEMV ops: the producer stores the chosen expert ids here
+  const float* gain;
+  float eps;
+  float* h_out;            // RESID_NORM: the op's task 0 stores h here
+  PSet src;                // NORM_SUM / SUM
+  int gstride;             // SUM: input offset per group
+  PSet gate, up;           // SWIGLU; slot j reads off + j * slot_stride
+  int slot_stride;
+  const float* am;         // COMBINE: attention partials (max, sum, weighted values)
+  const float* al;
+  const float* ao;
+  int nch, nheads, hdim;
+  // ---- attention
+  PSet qkv;       // dense: q|k|v projections; MLA: q_b output (q_pe is read from it)
+  PSet qlat;      // MLA: absorbed query [H * kv_lora]
+  PSet ckv;       // MLA: kv_a output (latent then RoPE key)
+  const float* kvnorm_g;
+  int hq, hkv, hd, gs;
+  int H, HG, kvl, rdim, nope;
+  void* kcache;   // dense: K of this layer [hkv][max_seq][hd]; MLA: [max_seq][kvl + rdim]
+  void* vcache;   // dense: V of this layer
+  int cache_bf16;
+  int max_seq;
+  const float* rope_cos;  // [max_seq][rope_dim / 2]
+  const float* rope_sin;
+  int rope_dim;
+  float attn_scale;
+  float* m_out;
+  float* l_out;
+  float* o_out;
+  int np;  // positions per ring stage
+  // ---- final op
+  const unsigned long long* fin_best;
+  int fin_n;
+  int vocab;
+  float* logits;  // LM head output (the final op reads nothing from it; kept for dumps)
+};
+
+struct StepState {
+  int epoch;  // 1-based step counter since the last reset (dependency counter targets)
+  int pos;    // position of the token of the current step
+  int tok;    // token of the current step (written by the host or by the previous step)
+  int last;   // greedy token of the last completed step
+};
+
+struct Status {
+  int code;  // 0 ok, 1 timeout
+  int cta, op, task;
+};
+
+struct KParams {
+  const OpDesc* ops;
+  int nops;
+  const int2* tasks;     // (op, task) pairs of all CTAs
+  const int* task_off;   // CTA b runs tasks[task_off[b] .. task_off[b + 1])
+  unsigned* counters;    // one per op, cumulative over steps
+  StepState* state;
+  unsigned* started;     // CTAs that have read the step state (cumulative)
+  Status* status;
+  unsigned long long timeout_ns;
+  int persistent;        // 1: one launch runs every op; 0: this launch runs op `op_only`
+  int op_only;
+  int n_ctas;
+  unsigned long long* trace;  // optional per-task timestamps
+  int trace_cap;
+  int tok_in;                 // >= 0: token of this step given by the host; < 0: the state's token
+};
+
+}  // namespace dec
