@@ -96,7 +96,10 @@ enum {
 /* dec_debug_dump selectors */
 #define DEC_DUMP_KV 1       /* dense: K then V, [n_layers][n_kv_heads][len][head_dim]; MLA: latent then pe */
 #define DEC_DUMP_ROUTES 2   /* MoE: int32 [n_moe_layers][top_k] expert ids of the last step */
-#define DEC_DUMP_TRACE 3    /* uint64 records {cta<<48|op<<32|task, t_wait, t_start, t_end} of the last step */
+#define DEC_DUMP_TRACE 3    /* uint64 records {cta<<48|op<<32|task, t_start, t_first_stage, t_done, t_published}
+                               (ns, %globaltimer) of every task of the last step */
+#define DEC_DUMP_TRACE_PRODUCER 6 /* uint64 pairs {cta<<48|op<<32|task, t_reached} per task-list position: when the
+                                     weight-streaming warp reached each task (ns) */
 #define DEC_DUMP_PLAN 4     /* text: one line per op (kind, tasks, geometry) */
 #define DEC_DUMP_WEIGHTS 5  /* bytes of weights read per step (uint64 x2: weights+scales, stored incl. padding) */
 #define DEC_DUMP_OP 100     /* + op index (DEC_DUMP_PLAN order): fp32 outputs of that op in the last step;

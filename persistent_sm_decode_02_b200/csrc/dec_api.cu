@@ -57,7 +57,10 @@ Geo gemv_geometry(int K, int wb) {
   const long long Kb = (long long)K * wb;
   int best = -1;
   long long best_waste = 1LL << 62;
-  for (int kcb = 4096; kcb >= 32; kcb >>= 1) {
+  // Prefer 512-byte row chunks: 32 lanes cover a row, so every row reduces
+  // inside one warp and tasks need no CTA-wide barrier; wider chunks only when
+  // 512 would pad K too much.
+  for (int kcb = 512; kcb >= 32; kcb >>= 1) {
     const long long pad = (Kb + kcb - 1) / kcb * kcb;
     const long long waste = pad - Kb;
     if (waste * 16 <= Kb) {
@@ -75,10 +78,7 @@ Geo gemv_geometry(int K, int wb) {
   g.nst_total = (int)(padb / best);
   g.cpr = best / 16;
   g.G = kConsumers / g.cpr;
-  int rpt = 8;
-  rpt = std::min(rpt, 128 / g.G);
-  rpt = std::min(rpt, kStageBytes / (g.G * best));
-  g.rpt = std::max(rpt, 1);
+  g.rpt = gemv_rows_per_thread(best);
   g.R = g.G * g.rpt;
   return g;
 }
@@ -156,6 +156,14 @@ __global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long lon
 
 __global__ void set_int(int* p, int v) { *p = v; }
 
+// One engine instance per (weight type, attention kind): each compiles only its own paths.
+const void* pick_kernel(int wtype, bool mla) {
+  if (mla) return wtype == WT_FP8 ? (const void*)engine_kernel<WT_FP8, true> : (const void*)engine_kernel<WT_BF16, true>;
+  if (wtype == WT_FP8) return (const void*)engine_kernel<WT_FP8, false>;
+  if (wtype == WT_BF16) return (const void*)engine_kernel<WT_BF16, false>;
+  return (const void*)engine_kernel<WT_F32, false>;
+}
+
 }  // namespace
 
 // ====================================================================== ctx
@@ -206,6 +214,7 @@ struct dec_ctx {
   uint8_t* staging = nullptr;
   size_t staging_bytes = 0;
   void* kvb_src = nullptr;
+  const void* kernel = nullptr;  // engine instance for this model's weight type and attention kind
   size_t weight_bytes_step = 0, weight_bytes_stored = 0;
 };
 
@@ -418,7 +427,10 @@ static int build_plan(dec_ctx* c) {
     }
   };
 
-  const int nch_dense = std::max(1, std::min(64, c->n_ctas / std::max(1, f.n_kv_heads)));
+  // split-KV chunks per head: about one attention task per CTA, at most 64 (one warp
+  // combines up to 64 chunks) and few enough that the combine weights fit the scratch
+  const int nch_dense = std::max(
+      1, std::min({64, c->n_ctas / std::max(1, f.n_kv_heads), kMaxCombine / std::max(1, f.n_heads)}));
   const int HG = kMlaHeadsPerTask;
   const int ngroups = mla ? (f.n_heads + HG - 1) / HG : 1;
   const int nch_mla = std::max(1, std::min(64, c->n_ctas / ngroups));
@@ -782,11 +794,26 @@ static int validate(const dec_config* f, dec_ctx* c) {
 }
 
 static int check_work_area(dec_ctx* c) {
+  // The prologues read partial sums with 16-byte loads: every vector they read
+  // must start, and every split must be strided, at a multiple of 4 floats.
+  auto al = [](const PSet& p) { return !p.ptr || (p.off % 4 == 0 && p.stride % 4 == 0); };
   for (size_t i = 0; i < c->ops.size(); ++i) {
     const OpDesc& o = c->ops[i];
-    if (o.kind == OP_GEMV && (long long)o.Kpad * (o.in_bf16 ? 2 : 4) > kWorkBytes)
-      return fail(c, DEC_ERR_UNSUPPORTED, "input vector of op %zu (%s) exceeds the work area", i,
-                  c->op_names[i].c_str());
+    const char* nm = c->op_names[i].c_str();
+    if (o.kind != OP_GEMV) continue;
+    const int cap = (o.pro == PRO_ATTN_COMBINE || o.pro == PRO_MLA_COMBINE) ? kCombineOff : kWorkBytes;
+    if ((long long)o.Kpad * (o.in_bf16 ? 2 : 4) > cap)
+      return fail(c, DEC_ERR_UNSUPPORTED, "input vector of op %zu (%s) exceeds the work area", i, nm);
+    if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.add2) || !al(o.routed) || !al(o.src) || !al(o.gate) ||
+        !al(o.up) || o.routed_slot_stride % 4 || o.slot_stride % 4 || o.gstride % 4 || o.hdim % 4)
+      return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): vector lengths and offsets must be multiples of 4", i, nm);
+    if ((o.pro == PRO_ATTN_COMBINE && (long long)o.nheads * o.nch > kMaxCombine) || o.nch > 64)
+      return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): too many split-KV chunks", i, nm);
+  }
+  for (size_t i = 0; i < c->ops.size(); ++i) {
+    const OpDesc& o = c->ops[i];
+    if (o.kind == OP_MLA && (o.qlat.stride % 4 || o.qlat.off % 4 || o.kvl % 4))
+      return fail(c, DEC_ERR_UNSUPPORTED, "MLA query layout must be a multiple of 4 floats");
   }
   return DEC_OK;
 }
@@ -821,9 +848,10 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
   int sms = 0, coop = 0;
   CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, f.device));
   CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, f.device));
-  CK(cudaFuncSetAttribute(engine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
+  c->kernel = pick_kernel(c->wtype, f.arch == DEC_ARCH_MLA_MOE);
+  CK(cudaFuncSetAttribute(c->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
   int per_sm = 0;
-  CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, engine_kernel, kThreads, kSmemBytes));
+  CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, c->kernel, kThreads, kSmemBytes));
   if (per_sm < 1 || !coop) return fail(c, DEC_ERR_UNSUPPORTED, "device cannot host the persistent kernel");
   c->n_ctas = f.n_ctas > 0 ? std::min(f.n_ctas, sms * per_sm) : sms;
   CK(cudaStreamCreateWithFlags(&c->stream, cudaStreamNonBlocking));
@@ -890,7 +918,7 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
     int total = 0;
     for (auto& o : c->ops) total += o.ntasks;
     c->trace_cap = total;
-    if ((rc = dalloc(c, &c->d_trace, (2 + 3 * (size_t)total) * 8))) return rc;
+    if ((rc = dalloc(c, &c->d_trace, (2 + 7 * (size_t)total) * 8))) return rc;
   }
   // bytes a step reads from the weight store (active weights + scales)
   for (auto& kv : c->mats) {
@@ -1177,8 +1205,8 @@ static int launch_per_op(dec_ctx* c, int tok_in) {
   for (int op = 0; op < (int)c->ops.size(); ++op) {
     KParams P = kparams(c, 0, op, op == 0 ? tok_in : -1);
     const int grid = std::min(c->ops[op].ntasks, c->n_ctas);
-    engine_kernel<<<grid, kThreads, kSmemBytes, c->stream>>>(P);
-    CK(cudaGetLastError());
+    void* args[] = {&P};
+    CK(cudaLaunchKernel(c->kernel, dim3(grid), dim3(kThreads), args, kSmemBytes, c->stream));
   }
   return DEC_OK;
 }
@@ -1210,13 +1238,12 @@ static int enqueue_step(dec_ctx* c, int32_t token_id) {
   if (token_id < 0 && c->epoch == 1)  // epoch 1: no step since the last reset / context install
     return fail(c, DEC_ERR_STATE, "no previous greedy token to feed back");
   CK(cudaSetDevice(f.device));
-  if (c->d_trace) CK(cudaMemsetAsync(c->d_trace, 0, 16, c->stream));
+  if (c->d_trace) CK(cudaMemsetAsync(c->d_trace, 0, (2 + 7 * (size_t)c->trace_cap) * 8, c->stream));
   int rc = DEC_OK;
   if (c->mode == DEC_PERSISTENT) {
     KParams P = kparams(c, 1, -1, token_id);
     void* args[] = {&P};
-    CK(cudaLaunchCooperativeKernel((const void*)engine_kernel, dim3(c->n_ctas), dim3(kThreads), args, kSmemBytes,
-                                   c->stream));
+    CK(cudaLaunchCooperativeKernel(c->kernel, dim3(c->n_ctas), dim3(kThreads), args, kSmemBytes, c->stream));
   } else if (c->mode == DEC_PER_OP) {
     rc = launch_per_op(c, token_id);
   } else {
@@ -1325,11 +1352,20 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     unsigned long long hdr[2];
     CK(cudaMemcpy(hdr, c->d_trace, 16, cudaMemcpyDeviceToHost));
     const size_t nrec = std::min<size_t>((unsigned)hdr[0], (size_t)c->trace_cap);
-    const size_t need = nrec * 24;
+    const size_t need = nrec * 40;
     if (out_bytes) *out_bytes = need;
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
     CK(cudaMemcpy(dst, c->d_trace + 2, need, cudaMemcpyDeviceToHost));
+    return DEC_OK;
+  }
+  if (what == DEC_DUMP_TRACE_PRODUCER) {
+    if (!c->d_trace) return fail(c, DEC_ERR_STATE, "context created without DEC_FLAG_TRACE");
+    const size_t need = (size_t)c->trace_cap * 16;
+    if (out_bytes) *out_bytes = need;
+    if (!dst) return DEC_OK;
+    if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
+    CK(cudaMemcpy(dst, c->d_trace + 2 + 5 * (size_t)c->trace_cap, need, cudaMemcpyDeviceToHost));
     return DEC_OK;
   }
   if (what == DEC_DUMP_PLAN) {

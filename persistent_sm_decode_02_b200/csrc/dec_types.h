@@ -14,16 +14,36 @@ namespace dec {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;  // threads that compute
-constexpr int kThreads = kConsumers + 32;        // + one producer warp that streams weights
+constexpr int kThreads = kConsumers + 64;        // + one producer warp (streams weights) + one signaller warp
 constexpr int kStageBytes = 32768;               // one ring stage
 constexpr int kStages = 5;                       // ring depth (160 KB in flight per SM)
 constexpr int kWorkBytes = 48 * 1024;            // per-task scratch (input vector / attention state)
+constexpr int kCombineOff = 40 * 1024;           // split-KV combine weights inside the scratch (<= 2048 floats)
+constexpr int kMaxCombine = (kWorkBytes - kCombineOff) / 4;
 constexpr int kMaxSegs = 20;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxD = 8192;                      // longest normalised vector (d_model, q_lora)
 constexpr int kMlaHeadsPerTask = 16;             // heads per CUDA-core MLA attention task
 
 enum WType : int { WT_F32 = 0, WT_BF16 = 1, WT_FP8 = 2 };
+
+// GEMV stage geometry, shared by the planner and the kernels: a stage holds
+// R = G * RPT rows of KCB bytes; each of the 256 consumer threads owns one
+// 16-byte column chunk (CPR = KCB / 16 chunks per row, G = 256 / CPR row
+// groups) of RPT rows; at most 128 rows (a tile never straddles a 128-row FP8
+// scale block) and at most one 32 KB stage.
+#ifdef __CUDACC__
+#define DEC_HD __host__ __device__
+#else
+#define DEC_HD
+#endif
+DEC_HD constexpr int gemv_rows_per_thread(int kcb) {
+  const int G = 256 / (kcb / 16);
+  int r = 8;
+  if (128 / G < r) r = 128 / G;
+  if (32768 / (G * kcb) < r) r = 32768 / (G * kcb);
+  return r < 1 ? 1 : r;
+}
 enum OpKind : int { OP_GEMV = 0, OP_ATTN = 1, OP_MLA = 2, OP_FINAL = 3 };
 enum Pro : int {
   PRO_NONE = 0,
@@ -54,7 +74,7 @@ struct Seg {
   int in_group;       // prologue input variant shared by all tasks of the segment (-1: by row group)
 };
 
-struct OpDesc {
+struct alignas(16) OpDesc {
   int kind, ntasks, layer;
   int dep[2];  // consumer dependencies (op index or -1)
   int pdep;    // producer dependency: router op whose top-k picks the weights of routed segments

@@ -1,16 +1,25 @@
 // Device engine of the decode step: tile tasks and the persistent scheduler.
 //
-// A CTA = 8 consumer warps (compute) + 1 producer warp (weight / KV streaming).
-// The producer walks the CTA's task list and streams every task's bytes from
-// HBM into a kStages-deep shared-memory ring with 1-D TMA bulk copies; it never
-// waits for activation dependencies (weights are static), so the next tasks'
-// weights are in flight while the consumers wait for the previous layer.  Only
-// routed-expert weights wait: their address comes from the router's top-k.
-// Consumers wait on the dependency counters of the task's op, build the
-// task's input vector in shared memory (norm / combine / SwiGLU prologue),
-// consume the ring stages and publish fp32 partial outputs plus one counter
-// increment.  Every wait is bounded by a global-timer deadline; on expiry the
-// CTA records the failure in a status word and drains its in-flight copies.
+// A CTA runs three warp roles:
+//   * 8 consumer warps compute the tasks;
+//   * 1 producer warp walks the CTA's task list and streams every task's bytes
+//     (weights, KV rows) from HBM into a kStages-deep shared-memory ring with
+//     1-D TMA bulk copies.  It never waits for activation dependencies
+//     (weights are static), so the next tasks' weights are in flight while
+//     the consumers wait for the previous layer; only routed-expert weights
+//     wait, because their address comes from the router's top-k;
+//   * 1 signaller warp publishes each finished task: it receives the task from
+//     the consumers through a two-slot mailbox guarded by mbarriers and does
+//     the gpu-scope fence and counter release, off the consumers' path.
+// Consumers wait on the dependency counters of the task's op (one thread polls,
+// then a barrier), build the task's input vector in shared memory (norm /
+// combine / SwiGLU prologue, once per op and input group), consume the ring
+// stages and write fp32 partial outputs.  Op descriptors are staged in shared
+// memory when the op changes; the next task-list entry is prefetched a task
+// ahead.  Every wait is bounded by a global-timer deadline: on expiry the CTA
+// records the failure in a status word, finishes the task it is in on stale
+// data (so that every thread meets the same barriers), stops, and drains the
+// copies still in flight.
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -20,28 +29,39 @@
 
 namespace dec {
 
+constexpr int kMail = 16;  // mailbox slots between consumers and the signaller
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kSignalWarp = kConsumerWarps + 1;
+constexpr int kOdBytes = (int)((sizeof(OpDesc) + 15) / 16 * 16);
+
 struct Misc {
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t sig_done[kMail];  // consumers -> signaller: task in mailbox slot finished (8 warp arrivals)
+  uint64_t sig_free[kMail];  // signaller -> consumers: mailbox slot published and free again
   StepState st;
   volatile int abort;
-  int x_op, x_group;   // identity of the input vector currently in the work area
-  int consumed;        // ring stages consumed (consumer thread 0)
-  int issued;          // ring stages issued (producer lane 0)
-  int prod_route_op;   // router op whose top-k is in prod_idx
+  int x_op, x_group;     // identity of the input vector currently in the work area
+  int consumed;          // ring stages consumed (consumer thread 0)
+  int issued;            // ring stages issued (producer lane 0)
+  int prod_route_op;     // router op whose top-k is in prod_idx
   int prod_idx[kMaxTopK];
   float cons_w[kMaxTopK];
+  int mail_op[kMail], mail_task[kMail];
+  unsigned long long mail_t[kMail][3];  // trace: task start, first stage available, compute done
+  unsigned long long tr_data;           // trace: when the current task's first stage was available
   float red[256];
   unsigned long long redk[8];
-  float attn_M[128], attn_den[128];
 };
 
 constexpr int kRingBytes = kStages * kStageBytes;
-constexpr int kSmemBytes = kRingBytes + kWorkBytes + (int)sizeof(Misc);
+constexpr int kSmemBytes = kRingBytes + kWorkBytes + 2 * kOdBytes + (int)sizeof(Misc);
 
 struct Smem {
   uint8_t* ring;
   uint8_t* work;
+  OpDesc* cod;  // consumers' copy of the current op descriptor
+  OpDesc* pod;  // producer's copy
   Misc* m;
 };
 
@@ -49,8 +69,17 @@ __device__ __forceinline__ Smem smem_layout(uint8_t* base) {
   Smem s;
   s.ring = base;
   s.work = base + kRingBytes;
-  s.m = reinterpret_cast<Misc*>(base + kRingBytes + kWorkBytes);
+  s.cod = reinterpret_cast<OpDesc*>(base + kRingBytes + kWorkBytes);
+  s.pod = reinterpret_cast<OpDesc*>(base + kRingBytes + kWorkBytes + kOdBytes);
+  s.m = reinterpret_cast<Misc*>(base + kRingBytes + kWorkBytes + 2 * kOdBytes);
   return s;
+}
+
+// Copy an op descriptor from global to shared memory (nthr threads with ids 0..nthr-1).
+__device__ __forceinline__ void copy_od(OpDesc* dst, const OpDesc* src, int id, int nthr) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  for (int i = id; i < kOdBytes / 16; i += nthr) d[i] = __ldg(s + i);
 }
 
 // ------------------------------------------------------------ error / waits
@@ -62,17 +91,21 @@ __device__ __forceinline__ void report_timeout(const KParams& P, int op, int tas
   }
 }
 
-// Spin until ready(); false if this CTA or another one gave up.
+// Spin until ready(); false if this CTA gave up (deadline passed or the CTA's
+// abort flag set).  Waits on another CTA (cross_cta) also watch the global status
+// word, so that a failure anywhere stops them; waits inside the CTA only read
+// the CTA's own flag (many threads spin on those: they must not load global
+// memory while they wait).
 template <class F>
 __device__ __forceinline__ bool bounded_wait(F ready, const KParams& P, volatile int* abort, int op, int task,
-                                             bool sleep) {
+                                             bool cross_cta) {
   if (ready()) return true;
   const uint64_t t0 = globaltimer();
   for (unsigned it = 1;; ++it) {
     if (ready()) return true;
-    if ((it & 31) == 0) {
+    if ((it & 63) == 0) {
       if (*abort) return false;
-      if (ld_volatile_int(&P.status->code) != 0) {
+      if (cross_cta && ld_volatile_int(&P.status->code) != 0) {
         *abort = 1;
         return false;
       }
@@ -82,16 +115,21 @@ __device__ __forceinline__ bool bounded_wait(F ready, const KParams& P, volatile
         return false;
       }
     }
-    if (sleep) __nanosleep(64);
+    if (cross_cta) __nanosleep(64);
   }
 }
 
 __device__ __forceinline__ bool wait_counter(const KParams& P, int dop, unsigned epoch, volatile int* abort,
                                              int op, int task) {
   if (dop < 0) return true;
-  const unsigned target = epoch * (unsigned)P.ops[dop].ntasks;
+  const unsigned target = epoch * (unsigned)__ldg(&P.ops[dop].ntasks);
   const unsigned* c = &P.counters[dop];
   return bounded_wait([&] { return (int)(ld_acquire_gpu(c) - target) >= 0; }, P, abort, op, task, true);
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t par, const KParams& P, volatile int* abort,
+                                          int op, int task) {
+  return bounded_wait([&] { return mbar_try_wait(bar, par); }, P, abort, op, task, false);
 }
 
 // ------------------------------------------------------- block reductions
@@ -126,6 +164,28 @@ __device__ __forceinline__ float pset(const PSet& p, int e) {
   return v;
 }
 
+__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+__device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
+  a.x = fmaf(w, b.x, a.x);
+  a.y = fmaf(w, b.y, a.y);
+  a.z = fmaf(w, b.z, a.z);
+  a.w = fmaf(w, b.w, a.w);
+}
+
+// Sum over splits of 4 consecutive elements (e multiple of 4, offsets 16-byte aligned).
+__device__ __forceinline__ float4 pset4(const PSet& p, int e) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* b = p.ptr + p.off + e;
+  for (int s = 0; s < p.S; ++s) add4(v, ldcg4(b + (size_t)s * p.stride));
+  return v;
+}
+
 __device__ __forceinline__ float rnd(float v, int bf16) { return bf16 ? bf16_round(v) : v; }
 
 __device__ __forceinline__ void store_x(uint8_t* work, int in_bf16, int e, float v) {
@@ -135,10 +195,23 @@ __device__ __forceinline__ void store_x(uint8_t* work, int in_bf16, int e, float
     reinterpret_cast<float*>(work)[e] = v;
 }
 
+// Four consecutive input elements (e multiple of 4), rounded to the input dtype.
+__device__ __forceinline__ void store_x4(uint8_t* work, int in_bf16, int e, float4 v) {
+  if (in_bf16) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(work + 2 * e) = u;
+  } else {
+    *reinterpret_cast<float4*>(work + 4 * e) = v;
+  }
+}
+
 // Softmax top-k router (one warp, all 32 lanes call): pick the k largest logits,
 // ties to the lower expert id, weights renormalised over the chosen k:
 // w_j = exp(r_j - r_max) / sum_i exp(r_i - r_max).
-__device__ void warp_route(const PSet& logits, int E, int k, int* idx_out, float* w_out) {
+__device__ __forceinline__ void warp_route(const PSet& logits, int E, int k, int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
   float v[8];
   int taken = 0;
@@ -169,7 +242,7 @@ __device__ void warp_route(const PSet& logits, int E, int k, int* idx_out, float
         bi = oi;
       }
     }
-    if (bi >= E) {  // only reachable with NaN logits: fall back to the lowest free id
+    if (bi >= E) {  // only reachable with NaN logits: fall back to id 0
       bi = 0;
       bv = -INFINITY;
     }
@@ -190,158 +263,200 @@ __device__ void warp_route(const PSet& logits, int E, int k, int* idx_out, float
 }
 
 // ------------------------------------------------------------- prologues
+// Every prologue reads its sources with 16-byte loads, several independent
+// loads in flight per thread, so it is bound by L2 bandwidth, not latency.
+constexpr int kMaxQ = kMaxD / 4 / kConsumers;  // float4 chunks per thread for vectors <= kMaxD
+
+// Split-KV log-sum-exp weights of one head: w_c = e^(m_c - M) / sum_c e^(m_c - M) l_c over
+// the chunks with data (l_c > 0), M = max m_c.  One warp; stores nch weights.
+__device__ __forceinline__ void combine_weights(const float* am, const float* al, int nch, float* w) {
+  const int lane = threadIdx.x & 31;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  if (lane < nch) {
+    l0 = ldcg(al + lane);
+    m0 = ldcg(am + lane);
+  }
+  if (lane + 32 < nch) {
+    l1 = ldcg(al + lane + 32);
+    m1 = ldcg(am + lane + 32);
+  }
+  const float M = warp_max(fmaxf(l0 > 0.f ? m0 : -INFINITY, l1 > 0.f ? m1 : -INFINITY));
+  const float e0 = l0 > 0.f ? expf(m0 - M) : 0.f, e1 = l1 > 0.f ? expf(m1 - M) : 0.f;
+  const float den = warp_sum(e0 * l0 + e1 * l1);
+  const float inv = den > 0.f ? 1.0f / den : 0.f;
+  if (lane < nch) w[lane] = e0 * inv;
+  if (lane + 32 < nch) w[lane + 32] = e1 * inv;
+}
+
 // Build the input vector of (op, group) in the work area, all 256 consumer threads.
-__device__ void prologue(const OpDesc& od, int group, int task, const Smem& S) {
+__device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, const Smem& S) {
   Misc* m = S.m;
   const int tid = threadIdx.x;
   uint8_t* x = S.work;
   const int n = od.n;
   const int bf = od.in_bf16;
   switch (od.pro) {
-    case PRO_RESID_NORM: {
-      if (od.routed.ptr) {
+    case PRO_RESID_NORM:
+    case PRO_NORM_SUM: {
+      const bool resid = od.pro == PRO_RESID_NORM;
+      if (resid && od.routed.ptr) {
         if (tid < 32) warp_route(od.route_logits, od.n_experts, od.top_k, nullptr, m->cons_w);
         named_bar_sync(1, kConsumers);
       }
-      constexpr int kPer = kMaxD / kConsumers;
-      float v[kPer];
-      float ss = 0.f;
+      float4 v[kMaxQ];
+      // base
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = tid + i * kConsumers;
-        float h = 0.f;
+      for (int i = 0; i < kMaxQ; ++i) {
+        const int e = 4 * (tid + i * kConsumers);
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (e < n) {
-          if (od.base_embed) {
+          if (!resid) {
+            v[i] = pset4(od.src, e);
+          } else if (od.base_embed) {
             const size_t row = (size_t)m->st.tok * n;
-            h = od.embed_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(od.embed)[row + e])
-                              : reinterpret_cast<const float*>(od.embed)[row + e];
-          } else {
-            h = ldcg(od.h_base + e);
-          }
-          if (od.add.ptr) h += pset(od.add, e);
-          if (od.routed.ptr) {
-            float r = 0.f;
-            for (int j = 0; j < od.top_k; ++j) {
-              PSet p = od.routed;
-              p.off += j * od.routed_slot_stride;
-              r += m->cons_w[j] * pset(p, e);
+            if (od.embed_bf16) {
+              const uint2 u = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(od.embed) + row + e));
+              v[i] = make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
+            } else {
+              v[i] = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(od.embed) + row + e));
             }
-            h += r;
+          } else {
+            v[i] = ldcg4(od.h_base + e);
           }
-          if (od.add2.ptr) h += pset(od.add2, e);
-          ss += h * h;
         }
-        v[i] = h;
       }
-      const float tot = consumer_sum(ss, m);
-      const float inv = 1.0f / sqrtf(tot / (float)n + od.eps);
+      if (resid) {
+        if (od.add.ptr) {
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = tid + i * kConsumers;
-        if (e < n) {
-          store_x(x, bf, e, rnd(v[i] * inv * od.gain[e], bf));
-          if (od.h_out && task == 0) od.h_out[e] = v[i];
+          for (int i = 0; i < kMaxQ; ++i) {
+            const int e = 4 * (tid + i * kConsumers);
+            if (e < n) add4(v[i], pset4(od.add, e));
+          }
+        }
+        if (od.add2.ptr) {
+#pragma unroll
+          for (int i = 0; i < kMaxQ; ++i) {
+            const int e = 4 * (tid + i * kConsumers);
+            if (e < n) add4(v[i], pset4(od.add2, e));
+          }
+        }
+        if (od.routed.ptr) {
+          for (int j = 0; j < od.top_k; ++j) {
+            PSet p = od.routed;
+            p.off += j * od.routed_slot_stride;
+            const float wj = m->cons_w[j];
+#pragma unroll
+            for (int i = 0; i < kMaxQ; ++i) {
+              const int e = 4 * (tid + i * kConsumers);
+              if (e < n) fma4(v[i], wj, pset4(p, e));
+            }
+          }
         }
       }
-      break;
-    }
-    case PRO_NORM_SUM: {
-      constexpr int kPer = kMaxD / kConsumers;
-      float v[kPer];
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = tid + i * kConsumers;
-        v[i] = e < n ? pset(od.src, e) : 0.f;
-        ss += v[i] * v[i];
-      }
+      for (int i = 0; i < kMaxQ; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
       const float tot = consumer_sum(ss, m);
       const float inv = 1.0f / sqrtf(tot / (float)n + od.eps);
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int e = tid + i * kConsumers;
-        if (e < n) store_x(x, bf, e, rnd(v[i] * inv * od.gain[e], bf));
+      for (int i = 0; i < kMaxQ; ++i) {
+        const int e = 4 * (tid + i * kConsumers);
+        if (e < n) {
+          const float4 g = __ldg(reinterpret_cast<const float4*>(od.gain + e));
+          float4 y;
+          y.x = v[i].x * inv * g.x;
+          y.y = v[i].y * inv * g.y;
+          y.z = v[i].z * inv * g.z;
+          y.w = v[i].w * inv * g.w;
+          store_x4(x, bf, e, y);
+          if (resid && od.h_out && task == 0) *reinterpret_cast<float4*>(od.h_out + e) = v[i];
+        }
       }
       break;
     }
     case PRO_SUM: {
       PSet p = od.src;
       p.off += group * od.gstride;
-      for (int e = tid; e < n; e += kConsumers) store_x(x, bf, e, rnd(pset(p, e), bf));
+      for (int e0 = 4 * tid; e0 < n; e0 += 4 * 4 * kConsumers) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * 4 * kConsumers;
+          if (e < n) v[u] = pset4(p, e);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * 4 * kConsumers;
+          if (e < n) store_x4(x, bf, e, v[u]);
+        }
+      }
       break;
     }
     case PRO_SWIGLU: {
-      PSet g = od.gate, u = od.up;
-      g.off += group * od.slot_stride;
-      u.off += group * od.slot_stride;
-      for (int e = tid; e < n; e += kConsumers) {
-        const float gv = pset(g, e), uv = pset(u, e);
-        store_x(x, bf, e, rnd(gv / (1.0f + expf(-gv)) * uv, bf));
+      PSet gp = od.gate, up = od.up;
+      gp.off += group * od.slot_stride;
+      up.off += group * od.slot_stride;
+      for (int e0 = 4 * tid; e0 < n; e0 += 4 * 4 * kConsumers) {
+        float4 gv[4], uv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * 4 * kConsumers;
+          if (e < n) {
+            gv[u] = pset4(gp, e);
+            uv[u] = pset4(up, e);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * 4 * kConsumers;
+          if (e < n) {
+            float4 y;
+            y.x = gv[u].x / (1.0f + expf(-gv[u].x)) * uv[u].x;
+            y.y = gv[u].y / (1.0f + expf(-gv[u].y)) * uv[u].y;
+            y.z = gv[u].z / (1.0f + expf(-gv[u].z)) * uv[u].z;
+            y.w = gv[u].w / (1.0f + expf(-gv[u].w)) * uv[u].w;
+            store_x4(x, bf, e, y);
+          }
+        }
       }
       break;
     }
-    case PRO_ATTN_COMBINE: {
-      // per head: M = max over chunks with data, den = sum e^(m_c - M) l_c
-      for (int h = tid; h < od.nheads; h += kConsumers) {
-        float M = -INFINITY;
-        for (int c = 0; c < od.nch; ++c)
-          if (ldcg(od.al + h * od.nch + c) > 0.f) M = fmaxf(M, ldcg(od.am + h * od.nch + c));
-        float den = 0.f;
-        for (int c = 0; c < od.nch; ++c) {
-          const float l = ldcg(od.al + h * od.nch + c);
-          if (l > 0.f) den += expf(ldcg(od.am + h * od.nch + c) - M) * l;
-        }
-        m->attn_M[h] = M;
-        m->attn_den[h] = den;
-      }
-      named_bar_sync(1, kConsumers);
-      for (int e = tid; e < n; e += kConsumers) {
-        const int h = e / od.hdim, d = e % od.hdim;
-        const float M = m->attn_M[h];
-        float num = 0.f;
-        for (int c = 0; c < od.nch; ++c) {
-          const float l = ldcg(od.al + h * od.nch + c);
-          if (l > 0.f) num += expf(ldcg(od.am + h * od.nch + c) - M) * ldcg(od.ao + ((size_t)h * od.nch + c) * od.hdim + d);
-        }
-        store_x(x, bf, e, rnd(num / m->attn_den[h], bf));
-      }
-      break;
-    }
+    case PRO_ATTN_COMBINE:
     case PRO_MLA_COMBINE: {
-      const int h = group;
-      if (tid < 32) {
-        float M = -INFINITY;
-        for (int c = tid; c < od.nch; c += 32)
-          if (ldcg(od.al + h * od.nch + c) > 0.f) M = fmaxf(M, ldcg(od.am + h * od.nch + c));
-        M = warp_max(M);
-        float den = 0.f;
-        for (int c = tid; c < od.nch; c += 32) {
-          const float l = ldcg(od.al + h * od.nch + c);
-          if (l > 0.f) den += expf(ldcg(od.am + h * od.nch + c) - M) * l;
-        }
-        den = warp_sum(den);
-        if (tid == 0) {
-          m->attn_M[0] = M;
-          m->attn_den[0] = den;
-        }
-      }
+      // per-chunk weights of every head this input needs, then weighted sums of the chunk outputs
+      const bool mla = od.pro == PRO_MLA_COMBINE;
+      const int h0 = mla ? group : 0, nh = mla ? 1 : od.nheads;
+      float* wt = reinterpret_cast<float*>(S.work + kCombineOff);  // [nh][nch]
+      const int warp = tid >> 5;
+      for (int h = warp; h < nh; h += kConsumerWarps)
+        combine_weights(od.am + (size_t)(h0 + h) * od.nch, od.al + (size_t)(h0 + h) * od.nch, od.nch,
+                        wt + h * od.nch);
       named_bar_sync(1, kConsumers);
-      const float M = m->attn_M[0], den = m->attn_den[0];
-      for (int e = tid; e < n; e += kConsumers) {
-        float num = 0.f;
-        for (int c = 0; c < od.nch; ++c) {
-          const float l = ldcg(od.al + h * od.nch + c);
-          if (l > 0.f) num += expf(ldcg(od.am + h * od.nch + c) - M) * ldcg(od.ao + ((size_t)h * od.nch + c) * od.hdim + e);
+      const int hd = od.hdim;
+      for (int e = 4 * tid; e < n; e += 4 * kConsumers) {
+        const int h = e / hd, d = e % hd;
+        const float* w = wt + h * od.nch;
+        const float* src = od.ao + ((size_t)(h0 + h) * od.nch) * hd + d;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int c = 0;
+        for (; c + 4 <= od.nch; c += 4) {
+          const float4 a0 = ldcg4(src + (size_t)c * hd), a1 = ldcg4(src + (size_t)(c + 1) * hd);
+          const float4 a2 = ldcg4(src + (size_t)(c + 2) * hd), a3 = ldcg4(src + (size_t)(c + 3) * hd);
+          fma4(acc, w[c], a0);
+          fma4(acc, w[c + 1], a1);
+          fma4(acc, w[c + 2], a2);
+          fma4(acc, w[c + 3], a3);
         }
-        store_x(x, bf, e, rnd(num / den, bf));
+        for (; c < od.nch; ++c) fma4(acc, w[c], ldcg4(src + (size_t)c * hd));
+        store_x4(x, bf, e, acc);
       }
       break;
     }
     default:
       break;
   }
-  // zero padding up to Kpad
-  for (int e = n + tid; e < od.Kpad; e += kConsumers) store_x(x, bf, e, 0.f);
+  // zero padding up to Kpad (n and Kpad are multiples of 4)
+  for (int e = n + 4 * tid; e < od.Kpad; e += 4 * kConsumers) store_x4(x, bf, e, make_float4(0.f, 0.f, 0.f, 0.f));
   named_bar_sync(1, kConsumers);
 }
 
@@ -363,10 +478,8 @@ __device__ __forceinline__ TaskGeo gemv_geo(const OpDesc& od, int t) {
   return g;
 }
 
-__device__ __forceinline__ bool wait_full(const KParams& P, const Smem& S, uint32_t g, int op, int task) {
-  uint64_t* bar = &S.m->full[g % kStages];
-  const uint32_t par = (g / kStages) & 1;
-  return bounded_wait([&] { return mbar_try_wait(bar, par); }, P, &S.m->abort, op, task, false);
+__device__ __forceinline__ void wait_full(const KParams& P, const Smem& S, uint32_t g, int op, int task) {
+  mbar_wait(&S.m->full[g % kStages], (g / kStages) & 1, P, &S.m->abort, op, task);
 }
 
 __device__ __forceinline__ void release_stage(const Smem& S, uint32_t g) {
@@ -381,7 +494,7 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
 }
 
 template <int WT>
-__device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* x, int k0, const OpDesc& od,
+__device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* x, int k0, int kcb, int G, int rpt,
                                            int c, int rg, float scale, float* acc) {
   if constexpr (WT == WT_FP8) {
     const uint4* xv = reinterpret_cast<const uint4*>(x + 2 * (k0 + c * 16));
@@ -395,9 +508,9 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (i >= od.rpt) break;
-      const int r = rg + od.G * i;
-      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * od.kcb + c * 16);
+      if (i >= rpt) break;
+      const int r = rg + G * i;
+      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * kcb + c * 16);
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
       float part = 0.f;
 #pragma unroll
@@ -422,9 +535,9 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (i >= od.rpt) break;
-      const int r = rg + od.G * i;
-      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * od.kcb + c * 16);
+      if (i >= rpt) break;
+      const int r = rg + G * i;
+      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * kcb + c * 16);
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
       float a = acc[i];
 #pragma unroll
@@ -438,9 +551,9 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
     const float4 xa = *reinterpret_cast<const float4*>(x + 4 * (k0 + c * 4));
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      if (i >= od.rpt) break;
-      const int r = rg + od.G * i;
-      const float4 wv = *reinterpret_cast<const float4*>(stage + r * od.kcb + c * 16);
+      if (i >= rpt) break;
+      const int r = rg + G * i;
+      const float4 wv = *reinterpret_cast<const float4*>(stage + r * kcb + c * 16);
       float a = acc[i];
       a = fmaf(wv.x, xa.x, a);
       a = fmaf(wv.y, xa.y, a);
@@ -451,68 +564,76 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
   }
 }
 
-template <int WT>
-__device__ bool gemv_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
-  const TaskGeo geo = gemv_geo(od, t);
+// One GEMV task, geometry fixed at compile time by the stage's bytes per row
+// (KCB): CPR 16-byte chunks per row, G row groups, RPT rows per thread.
+template <int WT, int KCB>
+__device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
+                                          uint32_t& g, const TaskGeo& geo) {
+  constexpr int CPR = KCB / 16, G = kConsumers / CPR, RPT = gemv_rows_per_thread(KCB), R = G * RPT;
+  constexpr int SPAN = CPR < 32 ? CPR : 32, PARTS = CPR / SPAN;
+  constexpr int KC = KCB / (WT == WT_FP8 ? 1 : WT == WT_BF16 ? 2 : 4);
   const Seg& sg = od.seg[geo.si];
   Misc* m = S.m;
-  if (m->x_op != op || m->x_group != geo.group) {
-    prologue(od, geo.group, t, S);
-    if (threadIdx.x == 0) {
-      m->x_op = op;
-      m->x_group = geo.group;
-    }
-  }
   const int tid = threadIdx.x;
-  const int c = tid % od.cpr, rg = tid / od.cpr;
-  float acc[8];
+  const int c = tid % CPR, rg = tid / CPR;
+  const int nst = od.nst;
+  float acc[RPT];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int i = 0; i < RPT; ++i) acc[i] = 0.f;
   const float* sc = nullptr;
   const int nkb = (od.K + 127) / 128;
-  for (int st = 0; st < od.nst; ++st) {
+  if constexpr (WT == WT_FP8) {
+    sc = sg.sc + (size_t)((geo.rt * R) / 128) * nkb;
+    if (sg.slot >= 0) sc += (size_t)m->prod_idx[sg.slot] * sg.s_estride;  // read after the first stage landed
+  }
+  for (int st = 0; st < nst; ++st) {
     wait_full(P, S, g, op, t);  // on failure the task runs to its end on stale data; the caller stops after it
+    if (P.trace && st == 0 && tid == 0) m->tr_data = globaltimer();
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    const int k0 = (geo.s * od.nst + st) * od.kc;
+    const int k0 = (geo.s * nst + st) * KC;
     float scale = 1.f;
     if constexpr (WT == WT_FP8) {
-      if (st == 0) {
-        sc = sg.sc + (size_t)((geo.rt * od.R) / 128) * nkb;
-        if (sg.slot >= 0) sc += (size_t)m->prod_idx[sg.slot] * sg.s_estride;
+      if (st == 0 && sg.slot >= 0) {  // the producer wrote the expert id before this stage's copy
+        sc = sg.sc + (size_t)((geo.rt * R) / 128) * nkb + (size_t)m->prod_idx[sg.slot] * sg.s_estride;
       }
       const int cb = (k0 + c * 16) >> 7;
       scale = cb < nkb ? __ldg(sc + cb) : 0.f;
     }
-    gemv_stage<WT>(stage, S.work, k0, od, c, rg, scale, acc);
+    gemv_stage<WT>(stage, S.work, k0, KCB, G, RPT, c, rg, scale, acc);
     release_stage(S, g);
     ++g;
   }
-  // reduce the cpr partials of every row
+  // reduce the CPR partials of every row
   const int lane = tid & 31, warp = tid >> 5;
-  const int span = od.cpr < 32 ? od.cpr : 32;
-  const int parts = od.cpr / span;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (i >= od.rpt) break;
-    float v = acc[i];
-    for (int o = span >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    acc[i] = v;
-  }
-  if ((lane & (span - 1)) == 0) {
-    const int part = od.cpr >= 32 ? (warp * 32 % od.cpr) / 32 : 0;
+  for (int o = SPAN >> 1; o > 0; o >>= 1)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i >= od.rpt) break;
-      m->red[(i * od.G + rg) * parts + part] = acc[i];
+    for (int i = 0; i < RPT; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  if (PARTS == 1 && !od.best) {
+    // a row's chunks all live in one warp: its first lane holds the row sum, no CTA barrier needed
+    if ((lane & (SPAN - 1)) == 0) {
+      float* out = od.out + (size_t)geo.s * od.out_stride + sg.out_off;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int row = geo.rt * R + rg + G * i;
+        if (row < sg.N) out[row] = acc[i];
+      }
     }
+    return;
+  }
+  if ((lane & (SPAN - 1)) == 0) {
+    const int part = CPR >= 32 ? (warp * 32 % CPR) / 32 : 0;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) m->red[(i * G + rg) * PARTS + part] = acc[i];
   }
   named_bar_sync(1, kConsumers);
   unsigned long long key = 0ull;
-  if (tid < od.R) {
-    const int i = tid / od.G, rg2 = tid % od.G;
+  if (tid < R) {
+    const int i = tid / G, rg2 = tid % G;
     float y = 0.f;
-    for (int p = 0; p < parts; ++p) y += m->red[(i * od.G + rg2) * parts + p];
-    const int row = geo.rt * od.R + tid;
+#pragma unroll
+    for (int p = 0; p < PARTS; ++p) y += m->red[(i * G + rg2) * PARTS + p];
+    const int row = geo.rt * R + tid;
     if (row < sg.N) {
       od.out[(size_t)geo.s * od.out_stride + sg.out_off + row] = y;
       if (od.best) key = argmax_key(y, sg.out_off + row);
@@ -532,7 +653,30 @@ __device__ bool gemv_consume(const KParams& P, const OpDesc& od, int op, int t, 
       od.best[t] = b;
     }
   }
-  return true;
+}
+
+template <int WT>
+__device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
+                                             uint32_t& g) {
+  const TaskGeo geo = gemv_geo(od, t);
+  Misc* m = S.m;
+  if (m->x_op != op || m->x_group != geo.group) {
+    prologue(od, geo.group, t, S);
+    if (threadIdx.x == 0) {
+      m->x_op = op;
+      m->x_group = geo.group;
+    }
+  }
+  switch (od.kcb) {
+    case 4096: gemv_task<WT, 4096>(P, od, op, t, S, g, geo); break;
+    case 2048: gemv_task<WT, 2048>(P, od, op, t, S, g, geo); break;
+    case 1024: gemv_task<WT, 1024>(P, od, op, t, S, g, geo); break;
+    case 512: gemv_task<WT, 512>(P, od, op, t, S, g, geo); break;
+    case 256: gemv_task<WT, 256>(P, od, op, t, S, g, geo); break;
+    case 128: gemv_task<WT, 128>(P, od, op, t, S, g, geo); break;
+    case 64: gemv_task<WT, 64>(P, od, op, t, S, g, geo); break;
+    default: gemv_task<WT, 32>(P, od, op, t, S, g, geo); break;
+  }
 }
 
 // ------------------------------------------------------- attention tasks
@@ -552,24 +696,20 @@ __device__ __forceinline__ ChunkB chunk_bounds(int c, int nch, int pos) {
   return b;
 }
 
-__device__ __forceinline__ int attn_stages(const OpDesc& od, int t, int pos) {
-  const int c = od.kind == OP_ATTN ? t % od.nch : t % od.nch;
-  const ChunkB b = chunk_bounds(c, od.nch, pos);
-  return (b.tc - b.t0 + od.np - 1) / od.np;
-}
-
 // Dense GQA split-KV attention: task = (kv head g, chunk c); all gs query heads of g.
 // Each head keeps a running (max m, sum l, weighted values o) over the chunk
 // (online softmax, Milakov & Gimelshein 2018) and publishes them for the
 // log-sum-exp combine in the output projection's prologue.
-__device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
+__device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kvh = t / od.nch, c = t % od.nch;
+  const int nch = od.nch, np = od.np;
+  const int kvh = t / nch, c = t % nch;
   const int pos = m->st.pos;
-  const ChunkB b = chunk_bounds(c, od.nch, pos);
-  const int hd = od.hd, gs = od.gs, cb = od.cache_bf16 ? 2 : 4;
+  const ChunkB b = chunk_bounds(c, nch, pos);
+  const int hd = od.hd, gs = od.gs, cbf = od.cache_bf16, cb = cbf ? 2 : 4;
   const int rowb = hd * cb;
+  const float scale = od.attn_scale;
   float* q_s = reinterpret_cast<float*>(S.work);           // [gs][hd]
   uint8_t* new_s = S.work + gs * hd * 4;                    // K row then V row (cache dtype)
   float* sc = reinterpret_cast<float*>(new_s + 2 * rowb);   // [gs][np]
@@ -581,17 +721,17 @@ __device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, 
     const int i = e / half, j = e % half;
     const int qh = kvh * gs + i;
     const float a = pset(od.qkv, qh * hd + j), bq = pset(od.qkv, qh * hd + j + half);
-    q_s[i * hd + j] = rnd(a * cosr[j] - bq * sinr[j], od.cache_bf16);
-    q_s[i * hd + j + half] = rnd(a * sinr[j] + bq * cosr[j], od.cache_bf16);
+    q_s[i * hd + j] = rnd(a * cosr[j] - bq * sinr[j], cbf);
+    q_s[i * hd + j + half] = rnd(a * sinr[j] + bq * cosr[j], cbf);
   }
   if (b.has_new) {
     const int koff = od.hq * hd + kvh * hd, voff = (od.hq + od.hkv) * hd + kvh * hd;
+    const size_t crow = ((size_t)kvh * od.max_seq + pos) * hd;
     for (int j = tid; j < half; j += kConsumers) {
       const float a = pset(od.qkv, koff + j), bk = pset(od.qkv, koff + j + half);
-      const float k0 = rnd(a * cosr[j] - bk * sinr[j], od.cache_bf16);
-      const float k1 = rnd(a * sinr[j] + bk * cosr[j], od.cache_bf16);
-      const size_t crow = ((size_t)kvh * od.max_seq + pos) * hd;
-      if (od.cache_bf16) {
+      const float k0 = rnd(a * cosr[j] - bk * sinr[j], cbf);
+      const float k1 = rnd(a * sinr[j] + bk * cosr[j], cbf);
+      if (cbf) {
         reinterpret_cast<__nv_bfloat16*>(new_s)[j] = __float2bfloat16_rn(k0);
         reinterpret_cast<__nv_bfloat16*>(new_s)[j + half] = __float2bfloat16_rn(k1);
         reinterpret_cast<__nv_bfloat16*>(od.kcache)[crow + j] = __float2bfloat16_rn(k0);
@@ -604,9 +744,8 @@ __device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, 
       }
     }
     for (int j = tid; j < hd; j += kConsumers) {
-      const float v = rnd(pset(od.qkv, voff + j), od.cache_bf16);
-      const size_t crow = ((size_t)kvh * od.max_seq + pos) * hd;
-      if (od.cache_bf16) {
+      const float v = rnd(pset(od.qkv, voff + j), cbf);
+      if (cbf) {
         reinterpret_cast<__nv_bfloat16*>(new_s + rowb)[j] = __float2bfloat16_rn(v);
         reinterpret_cast<__nv_bfloat16*>(od.vcache)[crow + j] = __float2bfloat16_rn(v);
       } else {
@@ -626,33 +765,34 @@ __device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, 
       const float* q = q_s + i * hd;
       const uint8_t* krow = Kp + (size_t)tt * rowb;
       float dot = 0.f;
+      int jj = tt % nck;
       for (int j = 0; j < nck; ++j) {
-        int jj = j + tt;
-        jj = jj % nck;
         const uint4 kv = *reinterpret_cast<const uint4*>(krow + jj * 16);
-        if (od.cache_bf16) {
-          const float* qq = q + jj * 8;
-          dot = fmaf(bf16lo(kv.x), qq[0], dot);
-          dot = fmaf(bf16hi(kv.x), qq[1], dot);
-          dot = fmaf(bf16lo(kv.y), qq[2], dot);
-          dot = fmaf(bf16hi(kv.y), qq[3], dot);
-          dot = fmaf(bf16lo(kv.z), qq[4], dot);
-          dot = fmaf(bf16hi(kv.z), qq[5], dot);
-          dot = fmaf(bf16lo(kv.w), qq[6], dot);
-          dot = fmaf(bf16hi(kv.w), qq[7], dot);
+        if (cbf) {
+          const float4 q0 = *reinterpret_cast<const float4*>(q + jj * 8);
+          const float4 q1 = *reinterpret_cast<const float4*>(q + jj * 8 + 4);
+          dot = fmaf(bf16lo(kv.x), q0.x, dot);
+          dot = fmaf(bf16hi(kv.x), q0.y, dot);
+          dot = fmaf(bf16lo(kv.y), q0.z, dot);
+          dot = fmaf(bf16hi(kv.y), q0.w, dot);
+          dot = fmaf(bf16lo(kv.z), q1.x, dot);
+          dot = fmaf(bf16hi(kv.z), q1.y, dot);
+          dot = fmaf(bf16lo(kv.w), q1.z, dot);
+          dot = fmaf(bf16hi(kv.w), q1.w, dot);
         } else {
-          const float* qq = q + jj * 4;
-          dot = fmaf(__uint_as_float(kv.x), qq[0], dot);
-          dot = fmaf(__uint_as_float(kv.y), qq[1], dot);
-          dot = fmaf(__uint_as_float(kv.z), qq[2], dot);
-          dot = fmaf(__uint_as_float(kv.w), qq[3], dot);
+          const float4 q0 = *reinterpret_cast<const float4*>(q + jj * 4);
+          dot = fmaf(__uint_as_float(kv.x), q0.x, dot);
+          dot = fmaf(__uint_as_float(kv.y), q0.y, dot);
+          dot = fmaf(__uint_as_float(kv.z), q0.z, dot);
+          dot = fmaf(__uint_as_float(kv.w), q0.w, dot);
         }
+        if (++jj == nck) jj = 0;
       }
-      sc[i * od.np + tt] = dot * od.attn_scale;
+      sc[i * np + tt] = dot * scale;
     }
     named_bar_sync(1, kConsumers);
     if (warp < gs) {
-      float* s = sc + warp * od.np;
+      float* s = sc + warp * np;
       float mx = -INFINITY;
       for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, s[tt]);
       mx = warp_max(mx);
@@ -672,7 +812,7 @@ __device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, 
       for (int tt = 0; tt < n; ++tt) {
         const float pv = s[tt];
         const uint8_t* vrow = Vp + (size_t)tt * rowb;
-        if (od.cache_bf16) {
+        if (cbf) {
           const __nv_bfloat16* vv = reinterpret_cast<const __nv_bfloat16*>(vrow) + lane * dpl;
           for (int d = 0; d < dpl; ++d) o[d] = fmaf(pv, __bfloat162float(vv[d]), o[d]);
         } else {
@@ -683,40 +823,41 @@ __device__ bool attn_consume(const KParams& P, const OpDesc& od, int op, int t, 
     }
     named_bar_sync(1, kConsumers);
   };
-  const int nst = (b.tc - b.t0 + od.np - 1) / od.np;
+  const int nst = (b.tc - b.t0 + np - 1) / np;
   for (int st = 0; st < nst; ++st) {
     wait_full(P, S, g, op, t);
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    const int a = b.t0 + st * od.np;
-    const int n = (b.tc - a) < od.np ? (b.tc - a) : od.np;
-    block(stage, stage + (size_t)od.np * rowb, n);
+    const int a = b.t0 + st * np;
+    const int n = (b.tc - a) < np ? (b.tc - a) : np;
+    block(stage, stage + (size_t)np * rowb, n);
     release_stage(S, g);
     ++g;
   }
   if (b.has_new) block(new_s, new_s + rowb, 1);
   if (warp < gs) {
     const int qh = kvh * gs + warp;
-    const size_t pi = (size_t)qh * od.nch + c;
+    const size_t pi = (size_t)qh * nch + c;
     if (lane == 0) {
       od.m_out[pi] = mrun;
       od.l_out[pi] = lrun;
     }
     for (int d = 0; d < dpl; ++d) od.o_out[pi * hd + lane * dpl + d] = o[d];
   }
-  return true;
 }
 
 // MLA absorbed-latent attention (CUDA cores): task = (head group of HG heads, chunk c).
 // s_h(t) = (q_lat^h . c_t + q_pe^h . kpe_t) * scale over the cached rows
 // [c_t | kpe_t]; the chunk holding position pos also normalises, RoPEs and
 // appends the new latent row (RMSNorm of the kv_a latent part, RoPE of its key part).
-__device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
+__device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hg = t / od.nch, c = t % od.nch;
-  const int HG = od.HG, kvl = od.kvl, rd = od.rdim, rowe = kvl + rd, rowb = rowe * 2;
+  const int nch = od.nch, np = od.np;
+  const int hg = t / nch, c = t % nch;
+  const int HG = od.HG, kvl = od.kvl, rd = od.rdim, rowe = kvl + rd, rowb = rowe * 2, H = od.H;
+  const float scale = od.attn_scale;
   const int pos = m->st.pos;
-  const ChunkB b = chunk_bounds(c, od.nch, pos);
+  const ChunkB b = chunk_bounds(c, nch, pos);
   float* ql = reinterpret_cast<float*>(S.work);            // [HG][kvl]
   float* qp = ql + HG * kvl;                                // [HG][rd]
   __nv_bfloat16* newrow = reinterpret_cast<__nv_bfloat16*>(qp + HG * rd);  // [rowe]
@@ -724,15 +865,22 @@ __device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, c
   const float* cosr = od.rope_cos + (size_t)pos * (rd / 2);
   const float* sinr = od.rope_sin + (size_t)pos * (rd / 2);
   const int h0 = hg * HG;
-  for (int e = tid; e < HG * kvl; e += kConsumers) {
+  // absorbed queries (rounded to bf16), 16-byte loads
+  for (int e = 4 * tid; e < HG * kvl; e += 4 * kConsumers) {
     const int i = e / kvl, j = e % kvl;
-    ql[e] = (h0 + i) < od.H ? bf16_round(pset(od.qlat, (h0 + i) * kvl + j)) : 0.f;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (h0 + i < H) v = pset4(od.qlat, (h0 + i) * kvl + j);
+    v.x = bf16_round(v.x);
+    v.y = bf16_round(v.y);
+    v.z = bf16_round(v.z);
+    v.w = bf16_round(v.w);
+    *reinterpret_cast<float4*>(ql + e) = v;
   }
   const int qstride = od.nope + rd;
   for (int e = tid; e < HG * (rd / 2); e += kConsumers) {
     const int i = e / (rd / 2), j = e % (rd / 2);
     float a = 0.f, bb = 0.f;
-    if (h0 + i < od.H) {
+    if (h0 + i < H) {
       a = pset(od.qkv, (h0 + i) * qstride + od.nope + j);
       bb = pset(od.qkv, (h0 + i) * qstride + od.nope + j + rd / 2);
     }
@@ -782,27 +930,28 @@ __device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, c
       const int i = p / n, tt = p % n;
       const uint8_t* row = rows + (size_t)tt * rowb;
       float dot = 0.f;
+      int jj = tt % nck;
       for (int j = 0; j < nck; ++j) {
-        int jj = j + tt;
-        jj = jj % nck;
         const uint4 kv = *reinterpret_cast<const uint4*>(row + jj * 16);
         const float* qq = jj < nql ? ql + i * kvl + jj * 8 : qp + i * rd + (jj - nql) * 8;
-        dot = fmaf(bf16lo(kv.x), qq[0], dot);
-        dot = fmaf(bf16hi(kv.x), qq[1], dot);
-        dot = fmaf(bf16lo(kv.y), qq[2], dot);
-        dot = fmaf(bf16hi(kv.y), qq[3], dot);
-        dot = fmaf(bf16lo(kv.z), qq[4], dot);
-        dot = fmaf(bf16hi(kv.z), qq[5], dot);
-        dot = fmaf(bf16lo(kv.w), qq[6], dot);
-        dot = fmaf(bf16hi(kv.w), qq[7], dot);
+        const float4 q0 = *reinterpret_cast<const float4*>(qq), q1 = *reinterpret_cast<const float4*>(qq + 4);
+        dot = fmaf(bf16lo(kv.x), q0.x, dot);
+        dot = fmaf(bf16hi(kv.x), q0.y, dot);
+        dot = fmaf(bf16lo(kv.y), q0.z, dot);
+        dot = fmaf(bf16hi(kv.y), q0.w, dot);
+        dot = fmaf(bf16lo(kv.z), q1.x, dot);
+        dot = fmaf(bf16hi(kv.z), q1.y, dot);
+        dot = fmaf(bf16lo(kv.w), q1.z, dot);
+        dot = fmaf(bf16hi(kv.w), q1.w, dot);
+        if (++jj == nck) jj = 0;
       }
-      sc[i * od.np + tt] = dot * od.attn_scale;
+      sc[i * np + tt] = dot * scale;
     }
     named_bar_sync(1, kConsumers);
 #pragma unroll
     for (int a = 0; a < 2; ++a) {
       if (a >= hpw) break;
-      float* s = sc + (warp * hpw + a) * od.np;
+      float* s = sc + (warp * hpw + a) * np;
       float mx = -INFINITY;
       for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, s[tt]);
       mx = warp_max(mx);
@@ -828,7 +977,7 @@ __device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, c
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
         if (a >= hpw) break;
-        const float pv = sc[(warp * hpw + a) * od.np + tt];
+        const float pv = sc[(warp * hpw + a) * np + tt];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           o[a][2 * q] = fmaf(pv, bf16lo(cw[q]), o[a][2 * q]);
@@ -838,12 +987,12 @@ __device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, c
     }
     named_bar_sync(1, kConsumers);
   };
-  const int nst = (b.tc - b.t0 + od.np - 1) / od.np;
+  const int nst = (b.tc - b.t0 + np - 1) / np;
   for (int st = 0; st < nst; ++st) {
     wait_full(P, S, g, op, t);
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    const int a = b.t0 + st * od.np;
-    const int n = (b.tc - a) < od.np ? (b.tc - a) : od.np;
+    const int a = b.t0 + st * np;
+    const int n = (b.tc - a) < np ? (b.tc - a) : np;
     block(stage, n);
     release_stage(S, g);
     ++g;
@@ -853,21 +1002,22 @@ __device__ bool mla_consume(const KParams& P, const OpDesc& od, int op, int t, c
   for (int a = 0; a < 2; ++a) {
     if (a >= hpw) break;
     const int h = h0 + warp * hpw + a;
-    if (h < od.H) {
-      const size_t pi = (size_t)h * od.nch + c;
+    if (h < H) {
+      const size_t pi = (size_t)h * nch + c;
       if (lane == 0) {
         od.m_out[pi] = mrun[a];
         od.l_out[pi] = lrun[a];
       }
+      float* dst = od.o_out + pi * kvl + lane * dpl;
 #pragma unroll
-      for (int d = 0; d < 16; ++d) od.o_out[pi * kvl + lane * dpl + d] = o[a][d];
+      for (int d = 0; d < 16; d += 4)
+        *reinterpret_cast<float4*>(dst + d) = make_float4(o[a][d], o[a][d + 1], o[a][d + 2], o[a][d + 3]);
     }
   }
-  return true;
 }
 
 // Final op: greedy token = argmax over the LM-head tasks' best keys; advance the step state.
-__device__ bool final_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S) {
+__device__ __forceinline__ void final_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S) {
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned long long key = 0ull;
@@ -901,32 +1051,37 @@ __device__ bool final_consume(const KParams& P, const OpDesc& od, int op, int t,
     ns.last = next;
     *P.state = ns;
   }
-  return true;
 }
 
 // ------------------------------------------------------------ task lists
+// Walks this CTA's (op, task) list; the entry after the current one is loaded a
+// task ahead so the list read never sits on the critical path.
 struct TaskIter {
-  const KParams* P;
-  int i, end, op, stride;
+  const int2* list;
+  int i, end, op, stride, persistent;
+  int2 nxt;
   __device__ void init(const KParams& p) {
-    P = &p;
-    if (p.persistent) {
+    persistent = p.persistent;
+    if (persistent) {
+      list = p.tasks;
       i = p.task_off[blockIdx.x];
       end = p.task_off[blockIdx.x + 1];
       stride = 1;
+      if (i < end) nxt = __ldg(list + i);
     } else {
+      list = nullptr;
       op = p.op_only;
       i = blockIdx.x;
-      end = p.ops[op].ntasks;
+      end = __ldg(&p.ops[op].ntasks);
       stride = gridDim.x;
     }
   }
   __device__ bool next(int& o, int& t) {
     if (i >= end) return false;
-    if (P->persistent) {
-      const int2 v = P->tasks[i];
-      o = v.x;
-      t = v.y;
+    if (persistent) {
+      o = nxt.x;
+      t = nxt.y;
+      if (i + 1 < end) nxt = __ldg(list + i + 1);
     } else {
       o = op;
       t = i;
@@ -945,15 +1100,16 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
   uint32_t g = 0;
   TaskIter it;
   it.init(P);
-  int op, t;
+  int op, t, cur = -1;
   const int pos = m->st.pos;
   const unsigned epoch = (unsigned)m->st.epoch;
+  const OpDesc& od = *S.pod;
   auto issue = [&](const void* src, uint32_t bytes, const void* src2, uint32_t bytes2, uint32_t off2,
                    uint64_t pol) -> bool {
     uint64_t* eb = &m->empty[g % kStages];
     const uint32_t par = ((g / kStages) & 1) ^ 1;
     int ready = 1;
-    if (lane == 0) ready = bounded_wait([&] { return mbar_try_wait(eb, par); }, P, &m->abort, op, t, false) ? 1 : 0;
+    if (lane == 0) ready = mbar_wait(eb, par, P, &m->abort, op, t) ? 1 : 0;
     if (!__shfl_sync(0xffffffffu, ready, 0)) return false;
     if (lane == 0) {
       uint8_t* dst = S.ring + (g % kStages) * kStageBytes;
@@ -968,7 +1124,19 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
   };
   bool ok = true;
   while (ok && it.next(op, t)) {
-    const OpDesc& od = P.ops[op];
+    if (op != cur) {
+      copy_od(S.pod, P.ops + op, lane, 32);
+      __syncwarp();
+      cur = op;
+    }
+    if (P.trace && lane == 0) {  // when the producer reached this task
+      const int idx = P.persistent ? it.i - 1 : t;
+      if (idx < P.trace_cap) {
+        unsigned long long* rec = P.trace + 2 + 5 * (size_t)P.trace_cap + 2 * (size_t)idx;
+        rec[0] = ((unsigned long long)blockIdx.x << 48) | ((unsigned long long)op << 32) | (unsigned)t;
+        rec[1] = globaltimer();
+      }
+    }
     if (od.kind == OP_GEMV) {
       const TaskGeo geo = gemv_geo(od, t);
       const Seg& sg = od.seg[geo.si];
@@ -1021,66 +1189,127 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
   if (lane == 0) m->issued = (int)g;
 }
 
-// --------------------------------------------------------------- consumer
-__device__ void consumer_loop(const KParams& P, const Smem& S) {
+// --------------------------------------------------------------- signaller
+// Hands a finished task (or the end sentinel op = -1) to the signaller warp.
+// Called by all consumer threads after the task's last barrier.
+__device__ __forceinline__ void post_task(const KParams& P, Misc* m, uint32_t q, int op, int t, uint64_t t0) {
+  const int slot = q % kMail;
+  const uint32_t par = (q / kMail) & 1;
+  if (threadIdx.x == 0) {
+    const uint64_t t_done = P.trace ? globaltimer() : 0;
+    mbar_wait(&m->sig_free[slot], par ^ 1, P, &m->abort, op, t);
+    m->mail_op[slot] = op;
+    m->mail_task[slot] = t;
+    m->mail_t[slot][0] = t0;
+    m->mail_t[slot][1] = m->tr_data;
+    m->mail_t[slot][2] = t_done;
+  }
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&m->sig_done[slot]);
+}
+
+// Publishes finished tasks in batches: it waits for the oldest unpublished task,
+// takes every later one that is already finished too, and releases the whole
+// batch with one gpu-scope fence and one counter add per run of equal ops.
+__device__ void signal_loop(const KParams& P, const Smem& S) {
   Misc* m = S.m;
-  uint32_t g = 0;
+  const int lane = threadIdx.x & 31;
+  uint32_t q = 0;
+  bool done = false;
+  while (!done) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait(&m->sig_done[q % kMail], (q / kMail) & 1, P, &m->abort, -1, (int)q) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    if (lane == 0) {
+      uint32_t end = q + 1;  // batch [q, end)
+      while (end - q < kMail && mbar_try_wait(&m->sig_done[end % kMail], (end / kMail) & 1)) ++end;
+      // every consumer write of these tasks happened before their mailbox hand-off
+      __threadfence();
+      uint32_t i = q;
+      while (i < end) {
+        const int op = m->mail_op[i % kMail];
+        if (op < 0) {
+          done = true;
+          end = i;
+          break;
+        }
+        uint32_t j = i + 1;
+        while (j < end && m->mail_op[j % kMail] == op) ++j;
+        red_release_gpu_add(&P.counters[op], j - i);
+        i = j;
+      }
+      if (P.trace) {
+        const uint64_t now = globaltimer();
+        const unsigned r0 = atomicAdd(reinterpret_cast<unsigned*>(P.trace), end - q);
+        for (uint32_t k = q; k < end; ++k) {
+          const unsigned r = r0 + (k - q);
+          if ((int)r < P.trace_cap) {
+            unsigned long long* rec = P.trace + 2 + (size_t)r * 5;
+            rec[0] = ((unsigned long long)blockIdx.x << 48) | ((unsigned long long)m->mail_op[k % kMail] << 32) |
+                     (unsigned)m->mail_task[k % kMail];
+            rec[1] = m->mail_t[k % kMail][0];
+            rec[2] = m->mail_t[k % kMail][1];
+            rec[3] = m->mail_t[k % kMail][2];
+            rec[4] = now;
+          }
+        }
+      }
+      for (uint32_t k = q; k < end; ++k) mbar_arrive(&m->sig_free[k % kMail]);
+      q = end;
+    }
+    done = __shfl_sync(0xffffffffu, done ? 1 : 0, 0) != 0;
+    q = __shfl_sync(0xffffffffu, q, 0);
+  }
+}
+
+// --------------------------------------------------------------- consumer
+// WT: weight storage type of the model; MLA: whether attention is the MLA kind.
+// Each model compiles only its own GEMV and attention paths.
+template <int WT, bool MLA>
+__device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
+  Misc* m = S.m;
+  uint32_t g = 0, q = 0;
   TaskIter it;
   it.init(P);
   int op, t, cur = -1;
   const unsigned epoch = (unsigned)m->st.epoch;
+  const OpDesc& od = *S.cod;
   while (it.next(op, t)) {
-    const OpDesc& od = P.ops[op];
     if (op != cur) {
+      copy_od(S.cod, P.ops + op, threadIdx.x, kConsumers);
       if (P.persistent && threadIdx.x == 0) {
-        if (wait_counter(P, od.dep[0], epoch, &m->abort, op, t)) wait_counter(P, od.dep[1], epoch, &m->abort, op, t);
+        const OpDesc* go = P.ops + op;
+        if (wait_counter(P, __ldg(&go->dep[0]), epoch, &m->abort, op, t))
+          wait_counter(P, __ldg(&go->dep[1]), epoch, &m->abort, op, t);
       }
       // uniform decision: every consumer thread sees the same value
       if (named_bar_or(1, kConsumers, m->abort)) break;
       cur = op;
     }
     const uint64_t t_start = P.trace ? globaltimer() : 0;
-    switch (od.kind) {
-      case OP_GEMV:
-        if (od.wtype == WT_FP8)
-          gemv_consume<WT_FP8>(P, od, op, t, S, g);
-        else if (od.wtype == WT_BF16)
-          gemv_consume<WT_BF16>(P, od, op, t, S, g);
-        else
-          gemv_consume<WT_F32>(P, od, op, t, S, g);
-        break;
-      case OP_ATTN:
-        attn_consume(P, od, op, t, S, g);
-        if (threadIdx.x == 0) m->x_op = -1;
-        break;
-      case OP_MLA:
+    if (P.trace && threadIdx.x == 0) m->tr_data = t_start;
+    const int kind = od.kind;
+    if (kind == OP_GEMV) {
+      gemv_consume<WT>(P, od, op, t, S, g);
+    } else if (kind == OP_FINAL) {
+      final_consume(P, od, op, t, S);
+    } else {
+      if constexpr (MLA)
         mla_consume(P, od, op, t, S, g);
-        if (threadIdx.x == 0) m->x_op = -1;
-        break;
-      case OP_FINAL:
-        final_consume(P, od, op, t, S);
-        break;
+      else
+        attn_consume(P, od, op, t, S, g);
+      if (threadIdx.x == 0) m->x_op = -1;
     }
     // A failed wait anywhere in the task makes every thread stop here, after the
     // task's barriers, without publishing the task.
     if (named_bar_or(1, kConsumers, m->abort)) break;
-    if (threadIdx.x == 0) {
-      __threadfence();
-      red_release_gpu_add(&P.counters[op], 1u);
-      if (P.trace) {
-        const int slot = atomicAdd(reinterpret_cast<unsigned*>(P.trace), 1u);
-        if (slot < P.trace_cap) {
-          unsigned long long* r = P.trace + 2 + (size_t)slot * 3;
-          r[0] = ((unsigned long long)blockIdx.x << 48) | ((unsigned long long)op << 32) | (unsigned)t;
-          r[1] = t_start;
-          r[2] = globaltimer();
-        }
-      }
-    }
+    post_task(P, m, q++, op, t, t_start);
   }
+  post_task(P, m, q, -1, -1, 0);  // end sentinel for the signaller
   if (threadIdx.x == 0) m->consumed = (int)g;
 }
 
+template <int WT, bool MLA>
 __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const Smem S = smem_layout(smem_raw);
@@ -1098,6 +1327,10 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
       mbar_init(&m->full[i], 1);
       mbar_init(&m->empty[i], kConsumerWarps);
     }
+    for (int i = 0; i < kMail; ++i) {
+      mbar_init(&m->sig_done[i], kConsumerWarps);
+      mbar_init(&m->sig_free[i], 1);
+    }
     fence_mbar_init();
     if (P.persistent) {
       __threadfence();
@@ -1105,10 +1338,13 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
     }
   }
   __syncthreads();
-  if (threadIdx.x >= kConsumers)
+  const int warp = threadIdx.x >> 5;
+  if (warp == kProducerWarp)
     producer_loop(P, S);
+  else if (warp == kSignalWarp)
+    signal_loop(P, S);
   else
-    consumer_loop(P, S);
+    consumer_loop<WT, MLA>(P, S);
   __syncthreads();
   // After a failure, let the copies still in flight land before the CTA exits.
   if (threadIdx.x == 0 && m->issued > m->consumed) {

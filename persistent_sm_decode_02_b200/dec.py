@@ -42,6 +42,7 @@ DEC_DUMP_ROUTES = 2
 DEC_DUMP_TRACE = 3
 DEC_DUMP_PLAN = 4
 DEC_DUMP_WEIGHTS = 5
+DEC_DUMP_TRACE_PRODUCER = 6
 DEC_DUMP_OP = 100
 
 EXPORTED = ["dec_create", "dec_load_weights", "dec_set_kv_cache", "dec_step", "dec_step_async", "dec_sync",
