@@ -180,9 +180,9 @@ __device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
 
 // Sum over splits of 4 consecutive elements (e multiple of 4, offsets 16-byte aligned).
 __device__ __forceinline__ float4 pset4(const PSet& p, int e) {
-  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* b = p.ptr + p.off + e;
-  for (int s = 0; s < p.S; ++s) add4(v, ldcg4(b + (size_t)s * p.stride));
+  float4 v = ldcg4(b);  // first split unconditionally, so callers' loads can be issued together
+  for (int s = 1; s < p.S; ++s) add4(v, ldcg4(b + (size_t)s * p.stride));
   return v;
 }
 
@@ -216,10 +216,26 @@ __device__ __forceinline__ void warp_route(const PSet& logits, int E, int k, int
   float v[8];
   int taken = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int e = lane + 32 * i;
-    v[i] = e < E ? pset(logits, e) : -INFINITY;
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  // sum the split-K partials, 4 splits x 8 logits = 32 independent loads per batch
+  const float* base = logits.ptr + logits.off;
+  for (int s0 = 0; s0 < logits.S; s0 += 4) {
+    float u[4][8];
+#pragma unroll
+    for (int ds = 0; ds < 4; ++ds)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        u[ds][i] = (s0 + ds < logits.S && e < E) ? ldcg(base + (size_t)(s0 + ds) * logits.stride + e) : 0.f;
+      }
+#pragma unroll
+    for (int ds = 0; ds < 4; ++ds)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += u[ds][i];
   }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (lane + 32 * i >= E) v[i] = -INFINITY;
   float top[kMaxTopK];
   int id[kMaxTopK];
   for (int j = 0; j < k; ++j) {
@@ -266,6 +282,7 @@ __device__ __forceinline__ void warp_route(const PSet& logits, int E, int k, int
 // Every prologue reads its sources with 16-byte loads, several independent
 // loads in flight per thread, so it is bound by L2 bandwidth, not latency.
 constexpr int kMaxQ = kMaxD / 4 / kConsumers;  // float4 chunks per thread for vectors <= kMaxD
+constexpr int kSrcBatch = 2;                    // residual sources loaded together
 
 // Split-KV log-sum-exp weights of one head: w_c = e^(m_c - M) / sum_c e^(m_c - M) l_c over
 // the chunks with data (l_c > 0), M = max m_c.  One warp; stores nch weights.
@@ -326,31 +343,42 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         }
       }
       if (resid) {
-        if (od.add.ptr) {
+        // Added sources: every split of `add` and `add2` (weight 1) and of each routed
+        // expert slot j (weight w_j).  kSrcBatch sources are loaded per batch so
+        // that each thread has up to kSrcBatch * kMaxQ 16-byte loads in flight.
+        const int na = od.add.ptr ? od.add.S : 0, nb = od.add2.ptr ? od.add2.S : 0;
+        const int nr = od.routed.ptr ? od.top_k * od.routed.S : 0;
+        const int nsrc = na + nb + nr;
+        auto src = [&](int k, float& wk) -> const float* {
+          wk = 1.f;
+          if (k < na) return od.add.ptr + od.add.off + (size_t)k * od.add.stride;
+          k -= na;
+          if (k < nb) return od.add2.ptr + od.add2.off + (size_t)k * od.add2.stride;
+          k -= nb;
+          const int j = k / od.routed.S, s = k % od.routed.S;
+          wk = m->cons_w[j];
+          return od.routed.ptr + od.routed.off + (size_t)j * od.routed_slot_stride + (size_t)s * od.routed.stride;
+        };
+        for (int k0 = 0; k0 < nsrc; k0 += kSrcBatch) {
+          float w3[kSrcBatch];
+          const float* p3[kSrcBatch];
+          float4 u[kSrcBatch][kMaxQ];
 #pragma unroll
-          for (int i = 0; i < kMaxQ; ++i) {
-            const int e = 4 * (tid + i * kConsumers);
-            if (e < n) add4(v[i], pset4(od.add, e));
+          for (int b = 0; b < kSrcBatch; ++b) {
+            p3[b] = k0 + b < nsrc ? src(k0 + b, w3[b]) : nullptr;
+            if (!p3[b]) w3[b] = 0.f;
           }
-        }
-        if (od.add2.ptr) {
 #pragma unroll
-          for (int i = 0; i < kMaxQ; ++i) {
-            const int e = 4 * (tid + i * kConsumers);
-            if (e < n) add4(v[i], pset4(od.add2, e));
-          }
-        }
-        if (od.routed.ptr) {
-          for (int j = 0; j < od.top_k; ++j) {
-            PSet p = od.routed;
-            p.off += j * od.routed_slot_stride;
-            const float wj = m->cons_w[j];
+          for (int b = 0; b < kSrcBatch; ++b)
 #pragma unroll
             for (int i = 0; i < kMaxQ; ++i) {
               const int e = 4 * (tid + i * kConsumers);
-              if (e < n) fma4(v[i], wj, pset4(p, e));
+              u[b][i] = (p3[b] && e < n) ? ldcg4(p3[b] + e) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-          }
+#pragma unroll
+          for (int b = 0; b < kSrcBatch; ++b)
+#pragma unroll
+            for (int i = 0; i < kMaxQ; ++i) fma4(v[i], w3[b], u[b][i]);  // w = 1: exact add
         }
       }
       float ss = 0.f;
