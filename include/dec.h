@@ -204,6 +204,39 @@ int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes, size_t* ou
 /* Text of the last error on this context (never NULL). */
 const char* dec_last_error(const dec_ctx* c);
 
+/* Split-KV decode attention for one query token that allocates no device
+ * memory.  The pages have no counterpart of this call; it exists for callers
+ * that cannot call cudaMalloc: code running while a CUDA graph is being
+ * captured, runtimes whose device memory belongs to an outside allocator that
+ * forbids allocation on the serving path, and embedders that must keep a fixed
+ * memory footprint once started.
+ *
+ * Computes, for every query head h (GQA: kv head = h / (n_heads/n_kv_heads)),
+ * out[h] = softmax_t(q[h] . K[g][t] / sqrt(head_dim)) V[g][t] over t < n_pos,
+ * split into position chunks whose (max, sum, weighted values) are combined
+ * with a log-sum-exp rescale -- the same split-KV attention the decode step
+ * runs.
+ *   q        device, fp32 [n_heads][head_dim] (already RoPE'd and rounded as wanted)
+ *   k_cache  device, bf16 [n_kv_heads][cache_stride][head_dim]
+ *   v_cache  device, bf16 [n_kv_heads][cache_stride][head_dim]
+ *   out      device, fp32 [n_heads][head_dim]
+ *   stream   cudaStream_t (NULL = legacy default stream); the call is asynchronous.
+ * Limits: head_dim 64 or 128, n_heads a multiple of n_kv_heads with at most 8
+ * query heads per kv head, 1 <= n_pos <= cache_stride, and the per-chunk
+ * partials n_heads * chunks * (head_dim + 2) floats must fit the library's
+ * fixed 2 MiB scratch (the call uses fewer chunks when needed and returns
+ * DEC_ERR_CAPACITY if even one chunk per head does not fit).
+ * The scratch is a fixed array inside the library, held by every GPU that
+ * loads it until the process exits, and shared by all calls: nothing in it has
+ * to start at zero (every call writes what it reads), but calls whose kernels
+ * overlap on the GPU (for example on two streams) race on it.  The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture.
+ * Errors: INVALID_ARG, CAPACITY, CUDA.  No context, no dec_last_error. */
+int dec_attention_noalloc(const float* q, const void* k_cache, const void* v_cache, int32_t n_heads,
+                          int32_t n_kv_heads, int32_t head_dim, int32_t n_pos, int32_t cache_stride, float* out,
+                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,7 +4,7 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "dec_api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "dec_api.cu"), os.path.join(HERE, "csrc", "noalloc.cu")]
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-Xcompiler", "-fPIC",
          "-shared", "-I", os.path.join(ROOT, "include")]
 

@@ -47,7 +47,7 @@ DEC_DUMP_OP = 100
 
 EXPORTED = ["dec_create", "dec_load_weights", "dec_set_kv_cache", "dec_step", "dec_step_async", "dec_sync",
             "dec_reset", "dec_destroy", "dec_set_stream", "dec_set_exec_mode", "dec_position", "dec_debug_dump",
-            "dec_last_error"]
+            "dec_last_error", "dec_attention_noalloc"]
 
 
 class dec_config(ctypes.Structure):
@@ -89,6 +89,8 @@ def load_library():
             "dec_set_exec_mode": [P, ctypes.c_int32],
             "dec_position": [P, ctypes.POINTER(ctypes.c_int32)],
             "dec_debug_dump": [P, ctypes.c_int32, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)],
+            "dec_attention_noalloc": [P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -166,6 +168,12 @@ def dec_debug_dump(ctx, what, dst, nbytes, out_bytes):
 
 def dec_last_error(ctx):
     return load_library().dec_last_error(ctx).decode()
+
+
+def dec_attention_noalloc(q, k_cache, v_cache, n_heads, n_kv_heads, head_dim, n_pos, cache_stride, out, stream):
+    """Allocation-free split-KV attention (device addresses in, status code out); see include/dec.h."""
+    return load_library().dec_attention_noalloc(q, k_cache, v_cache, n_heads, n_kv_heads, head_dim, n_pos,
+                                                cache_stride, out, stream)
 
 
 # ---- convenience
