@@ -60,6 +60,8 @@ extern "C" {
 #define DEC_PER_OP_GRAPH 2 /* same tiles, one kernel per op, replayed from a CUDA graph */
 
 #define DEC_FLAG_TRACE 1u /* record per-task timestamps (dec_debug_dump DEC_DUMP_TRACE) */
+#define DEC_FLAG_TEST_STALL 2u /* failure-path test: the first task of the first op is never published, so
+                                  the persistent kernel's dependency waits run out (DEC_ERR_TIMEOUT) */
 
 /* Weight kinds for dec_tensor.kind.  Layouts are row-major [rows][cols]; FP8
  * matrices carry scales [ceil(rows/128)][ceil(cols/128)] fp32; norm gains are

@@ -646,7 +646,7 @@ static int build_plan(dec_ctx* c) {
         segs.push_back({sg, -1, 0});
         segs.push_back({su, -1, 0});
       }
-      int egu = P.gemv(segs, d, l, false, "experts gate|up");
+      int egu = P.gemv(segs, d, l, false, "exp_gate|up");
       if (egu < 0) return P.rc;
       const OpDesc& rop = c->ops[ro];
       const PSet rlog{rop.out, rop.S, rop.out_stride, 0};
@@ -666,7 +666,7 @@ static int build_plan(dec_ctx* c) {
         sd = P.new_mat(DEC_W_SH_DOWN, l, d, eh * f.n_shared, 1, 0);
         dsegs.push_back({sd, -1, k});
       }
-      int edn = P.gemv(dsegs, eh, l, false, "experts down");
+      int edn = P.gemv(dsegs, eh, l, false, "exp_down");
       if (edn < 0) return P.rc;
       {
         OpDesc& o = c->ops[edn];
@@ -1198,6 +1198,7 @@ static KParams kparams(dec_ctx* c, int persistent, int op, int tok_in) {
   P.trace = c->d_trace;
   P.trace_cap = c->trace_cap;
   P.tok_in = tok_in;
+  P.test_stall = (c->cfg.flags & DEC_FLAG_TEST_STALL) ? 1 : 0;
   return P;
 }
 

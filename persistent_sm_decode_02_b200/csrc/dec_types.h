@@ -165,6 +165,7 @@ struct KParams {
   unsigned long long* trace;  // optional per-task timestamps
   int trace_cap;
   int tok_in;                 // >= 0: token of this step given by the host; < 0: the state's token
+  int test_stall;             // failure-path test: never publish task 0 of op 0
 };
 
 }  // namespace dec

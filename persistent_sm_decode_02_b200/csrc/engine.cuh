@@ -1263,7 +1263,11 @@ __device__ void signal_loop(const KParams& P, const Smem& S) {
         }
         uint32_t j = i + 1;
         while (j < end && m->mail_op[j % kMail] == op) ++j;
-        red_release_gpu_add(&P.counters[op], j - i);
+        uint32_t cnt = j - i;
+        if (P.test_stall && op == 0)  // failure-path test: task 0 of op 0 is never published
+          for (uint32_t z = i; z < j; ++z)
+            if (m->mail_task[z % kMail] == 0) --cnt;
+        if (cnt) red_release_gpu_add(&P.counters[op], cnt);
         i = j;
       }
       if (P.trace) {

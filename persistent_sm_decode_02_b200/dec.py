@@ -32,6 +32,7 @@ DEC_PERSISTENT = 0
 DEC_PER_OP = 1
 DEC_PER_OP_GRAPH = 2
 DEC_FLAG_TRACE = 1
+DEC_FLAG_TEST_STALL = 2
 
 DEC_W = dict(embed=1, final_norm=2, lm_head=3, attn_norm=10, wq=11, wk=12, wv=13, wo=14, ffn_norm=15,
              w_gate=16, w_up=17, w_down=18, q_a=20, q_a_norm=21, q_b=22, kv_a=23, kv_a_norm=24, kv_b=25,
