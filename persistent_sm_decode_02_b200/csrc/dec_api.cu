@@ -156,6 +156,22 @@ __global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long lon
 
 __global__ void set_int(int* p, int v) { *p = v; }
 
+// Row-major latent rows [n][rowe] (bf16) <-> the blocked tensor-core cache layout
+// (mla_cache_off); one thread per 16-byte chunk.
+__global__ void mla_cache_convert(uint8_t* rows, uint8_t* blocked, int n, int rowe, int to_blocked) {
+  const long long nck = rowe / 8, total = (long long)n * nck;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int p = (int)(i / nck), k = (int)(i % nck);
+    uint4* r = reinterpret_cast<uint4*>(rows + (size_t)p * rowe * 2 + (size_t)k * 16);
+    uint4* b = reinterpret_cast<uint4*>(blocked + (size_t)(p / kMlaBlock) * rowe * kMlaBlock * 2 +
+                                        mla_cache_off(p % kMlaBlock, 8 * k));
+    if (to_blocked)
+      *b = *r;
+    else
+      *r = *b;
+  }
+}
+
 // One engine instance per (weight type, attention kind): each compiles only its own paths.
 const void* pick_kernel(int wtype, bool mla) {
   if (mla) return wtype == WT_FP8 ? (const void*)engine_kernel<WT_FP8, true> : (const void*)engine_kernel<WT_BF16, true>;
@@ -375,6 +391,10 @@ static int alloc_mats(dec_ctx* c) {
   return DEC_OK;
 }
 
+static size_t mla_cache_bytes(const dec_config& f) {
+  return (size_t)((f.max_seq + kMlaBlock - 1) / kMlaBlock) * kMlaBlock * (f.kv_lora + f.qk_rope) * 2;
+}
+
 static float* gainp(dec_ctx* c, int kind, int layer) { return c->vecs[{kind, layer}].p; }
 
 static int build_plan(dec_ctx* c) {
@@ -431,9 +451,8 @@ static int build_plan(dec_ctx* c) {
   // combines up to 64 chunks) and few enough that the combine weights fit the scratch
   const int nch_dense = std::max(
       1, std::min({64, c->n_ctas / std::max(1, f.n_kv_heads), kMaxCombine / std::max(1, f.n_heads)}));
-  const int HG = kMlaHeadsPerTask;
-  const int ngroups = mla ? (f.n_heads + HG - 1) / HG : 1;
-  const int nch_mla = std::max(1, std::min(64, c->n_ctas / ngroups));
+  // MLA: one attention task per cache block of kMlaBlock positions
+  const int nch_mla = (f.max_seq + kMlaBlock - 1) / kMlaBlock;
   c->n_moe = 0;
 
   for (int l = 0; l < L; ++l) {
@@ -518,8 +537,15 @@ static int build_plan(dec_ctx* c) {
         o.dep[0] = s1;
       }
       Mat* uk = P.new_mat(DEC_W_KV_B * 16 + 1, l, H * kvl, nope, 1, 1);  // W_UK^T view of kv_b
-      int s3 = P.gemv({{uk, -1, -1}}, nope, l, false, "absorb_q");
+      int s3 = P.gemv({{uk, -1, -1}}, nope, l, true, "absorb_q");
       if (s3 < 0) return P.rc;
+      // bf16 absorbed query [q_lat | q_pe] of all kMlaHeads (zero-padded) in the tensor-core layout
+      void* qc = nullptr;
+      {
+        const size_t qb = (size_t)(kvl + rd) / 8 * 2048;
+        if (dalloc(c, reinterpret_cast<uint8_t**>(&qc), qb)) return DEC_ERR_OOM;
+        CK(cudaMemsetAsync(qc, 0, qb, c->stream));
+      }
       {
         OpDesc& o = c->ops[s3];
         const OpDesc& p = c->ops[s2];
@@ -529,31 +555,33 @@ static int build_plan(dec_ctx* c) {
         o.gstride = nope + rd;
         o.rows_per_group = kvl;
         o.dep[0] = s2;
+        o.qc = qc;
+        o.nope = nope;
+        o.rdim = rd;
+        o.rope_cos = c->rope_cos;
+        o.rope_sin = c->rope_sin;
       }
       OpDesc a = P.base_op(OP_MLA, l);
       {
         const OpDesc& p1 = c->ops[s1];
-        const OpDesc& p2 = c->ops[s2];
-        const OpDesc& p3 = c->ops[s3];
         a.H = H;
-        a.HG = HG;
         a.kvl = kvl;
         a.rdim = rd;
         a.nope = nope;
         a.nch = nch_mla;
-        a.ntasks = ngroups * a.nch;
-        a.qkv = PSet{p2.out, p2.S, p2.out_stride, 0};
-        a.qlat = PSet{p3.out, p3.S, p3.out_stride, 0};
+        a.ntasks = nch_mla;
+        a.qc = qc;
         a.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
         a.dep[0] = s3;
+        a.pdep = s3;  // the producer streams the absorbed query
         a.max_seq = f.max_seq;
         a.cache_bf16 = 1;
         a.rope_dim = rd;
         a.attn_scale = (float)(1.0 / std::sqrt((double)(nope + rd)));
-        a.np = kStageBytes / ((kvl + rd) * 2);
         for (int i = 0; i < 3; ++i) {
           size_t n = (size_t)H * a.nch * (i == 2 ? kvl : 1);
           if (dalloc(c, &attn_buf[i], n * 4)) return DEC_ERR_OOM;
+          CK(cudaMemsetAsync(attn_buf[i], 0, n * 4, c->stream));
         }
         a.m_out = attn_buf[0];
         a.l_out = attn_buf[1];
@@ -774,8 +802,10 @@ static int validate(const dec_config* f, dec_ctx* c) {
     if (!k_ok((long long)f->n_heads * f->head_dim)) return uns("n_heads*head_dim alignment");
   } else {
     if (f->weight_dtype == DEC_F32) return uns("MLA needs bf16 activations (bf16 or fp8 weights)");
+    // tensor-core attention: heads fill (at most) the MMA's 128 rows; 64-dim K chunks; 256-dim O halves
     if (f->kv_lora != 512) return uns("kv_lora must be 512");
-    if (f->qk_rope < 16 || f->qk_rope > 128 || f->qk_rope % 16) return uns("qk_rope");
+    if (f->qk_rope != 64 && f->qk_rope != 128) return uns("qk_rope must be 64 or 128");
+    if (f->n_heads > kMlaHeads) return uns("MLA n_heads > 128");
     if (f->qk_nope < 16 || !k_ok(f->qk_nope)) return uns("qk_nope");
     if (f->v_head < 8 || !k_ok((long long)f->n_heads * f->v_head)) return uns("v_head");
     if (f->n_heads < 1 || f->n_heads > 1024) return bad("n_heads");
@@ -807,13 +837,9 @@ static int check_work_area(dec_ctx* c) {
     if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.add2) || !al(o.routed) || !al(o.src) || !al(o.gate) ||
         !al(o.up) || o.routed_slot_stride % 4 || o.slot_stride % 4 || o.gstride % 4 || o.hdim % 4)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): vector lengths and offsets must be multiples of 4", i, nm);
-    if ((o.pro == PRO_ATTN_COMBINE && (long long)o.nheads * o.nch > kMaxCombine) || o.nch > 64)
+    if ((o.pro == PRO_ATTN_COMBINE && (o.nch > 64 || (long long)o.nheads * o.nch > kMaxCombine)) ||
+        (o.pro == PRO_MLA_COMBINE && o.nch > kMaxCombine))
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): too many split-KV chunks", i, nm);
-  }
-  for (size_t i = 0; i < c->ops.size(); ++i) {
-    const OpDesc& o = c->ops[i];
-    if (o.kind == OP_MLA && (o.qlat.stride % 4 || o.qlat.off % 4 || o.kvl % 4))
-      return fail(c, DEC_ERR_UNSUPPORTED, "MLA query layout must be a multiple of 4 floats");
   }
   return DEC_OK;
 }
@@ -878,8 +904,8 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
       if ((rc = dalloc(c, reinterpret_cast<uint8_t**>(&c->vc[l]), n))) return rc;
       CK(cudaMemsetAsync(c->kc[l], 0, n, c->stream));
       CK(cudaMemsetAsync(c->vc[l], 0, n, c->stream));
-    } else {
-      const size_t n = (size_t)f.max_seq * (f.kv_lora + f.qk_rope) * 2;
+    } else {  // whole blocks, zeroed: an MMA reads the unused tail rows of the last block (with P = 0)
+      const size_t n = mla_cache_bytes(f);
       if ((rc = dalloc(c, reinterpret_cast<uint8_t**>(&c->kc[l]), n))) return rc;
       CK(cudaMemsetAsync(c->kc[l], 0, n, c->stream));
     }
@@ -1153,6 +1179,7 @@ extern "C" int dec_set_kv_cache(dec_ctx* c, const void* k_or_latent, const void*
   int rc = dec_reset(c);
   if (rc) return rc;
   const bool mla = f.arch == DEC_ARCH_MLA_MOE;
+  uint8_t* rows = nullptr;
   for (int l = 0; l < f.n_layers && n_tokens > 0; ++l) {
     if (!mla) {
       const size_t row = (size_t)n_tokens * f.head_dim * c->eb;  // one kv head
@@ -1162,13 +1189,26 @@ extern "C" int dec_set_kv_cache(dec_ctx* c, const void* k_or_latent, const void*
                            cudaMemcpyDefault, c->stream));
       CK(cudaMemcpy2DAsync(c->vc[l], dpitch, (const uint8_t*)v_or_pe + l * src_layer, row, row, f.n_kv_heads,
                            cudaMemcpyDefault, c->stream));
-    } else {
+    } else {  // rows [n][kv_lora | qk_rope] in a scratch buffer, then the blocked layout
       const size_t lat = (size_t)f.kv_lora * 2, pe = (size_t)f.qk_rope * 2, rowb = lat + pe;
-      CK(cudaMemcpy2DAsync(c->kc[l], rowb, (const uint8_t*)k_or_latent + (size_t)l * n_tokens * lat, lat, lat,
-                           n_tokens, cudaMemcpyDefault, c->stream));
-      CK(cudaMemcpy2DAsync((uint8_t*)c->kc[l] + lat, rowb, (const uint8_t*)v_or_pe + (size_t)l * n_tokens * pe, pe, pe,
-                           n_tokens, cudaMemcpyDefault, c->stream));
+      if (!rows) {
+        cudaError_t e = cudaMalloc(&rows, (size_t)n_tokens * rowb);
+        if (e != cudaSuccess) {
+          (void)cudaGetLastError();
+          return fail(c, DEC_ERR_OOM, "cache scratch of %zu bytes: %s", (size_t)n_tokens * rowb, cudaGetErrorString(e));
+        }
+      }
+      CK(cudaMemcpy2DAsync(rows, rowb, (const uint8_t*)k_or_latent + (size_t)l * n_tokens * lat, lat, lat, n_tokens,
+                           cudaMemcpyDefault, c->stream));
+      CK(cudaMemcpy2DAsync(rows + lat, rowb, (const uint8_t*)v_or_pe + (size_t)l * n_tokens * pe, pe, pe, n_tokens,
+                           cudaMemcpyDefault, c->stream));
+      mla_cache_convert<<<1184, 256, 0, c->stream>>>(rows, (uint8_t*)c->kc[l], n_tokens, f.kv_lora + f.qk_rope, 1);
+      CK(cudaGetLastError());
     }
+  }
+  if (rows) {
+    CK(cudaStreamSynchronize(c->stream));
+    CK(cudaFree(rows));
   }
   StepState st{1, n_tokens, 0, 0};
   CK(cudaMemcpyAsync(c->d_state, &st, sizeof st, cudaMemcpyHostToDevice, c->stream));
@@ -1324,6 +1364,7 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
     uint8_t* o = reinterpret_cast<uint8_t*>(dst);
+    uint8_t* rows = nullptr;
     for (int l = 0; l < f.n_layers && n > 0; ++l) {
       if (!mla) {
         const size_t row = (size_t)n * f.head_dim * c->eb, sp = (size_t)f.max_seq * f.head_dim * c->eb;
@@ -1333,11 +1374,21 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
       } else {
         const size_t lat = (size_t)f.kv_lora * 2, pe = (size_t)f.qk_rope * 2, rowb = lat + pe;
         const size_t nl = (size_t)f.n_layers * n;
-        CK(cudaMemcpy2D(o + (size_t)l * n * lat, lat, c->kc[l], rowb, lat, n, cudaMemcpyDeviceToHost));
-        CK(cudaMemcpy2D(o + nl * lat + (size_t)l * n * pe, pe, (uint8_t*)c->kc[l] + lat, rowb, pe, n,
-                        cudaMemcpyDeviceToHost));
+        if (!rows) {
+          cudaError_t e = cudaMalloc(&rows, (size_t)n * rowb);
+          if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return fail(c, DEC_ERR_OOM, "dump scratch: %s", cudaGetErrorString(e));
+          }
+        }
+        mla_cache_convert<<<1184, 256, 0, c->stream>>>(rows, (uint8_t*)c->kc[l], n, f.kv_lora + f.qk_rope, 0);
+        CK(cudaGetLastError());
+        CK(cudaStreamSynchronize(c->stream));
+        CK(cudaMemcpy2D(o + (size_t)l * n * lat, lat, rows, rowb, lat, n, cudaMemcpyDeviceToHost));
+        CK(cudaMemcpy2D(o + nl * lat + (size_t)l * n * pe, pe, rows + lat, rowb, pe, n, cudaMemcpyDeviceToHost));
       }
     }
+    if (rows) CK(cudaFree(rows));
     return DEC_OK;
   }
   if (what == DEC_DUMP_ROUTES) {

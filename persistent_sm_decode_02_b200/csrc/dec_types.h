@@ -23,7 +23,8 @@ constexpr int kMaxCombine = (kWorkBytes - kCombineOff) / 4;
 constexpr int kMaxSegs = 20;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxD = 8192;                      // longest normalised vector (d_model, q_lora)
-constexpr int kMlaHeadsPerTask = 16;             // heads per CUDA-core MLA attention task
+constexpr int kMlaHeads = 128;                   // MLA attention: heads are the MMA's M dimension (zero-padded)
+constexpr int kMlaBlock = 64;                    // MLA attention: cache positions per block and per task
 
 enum WType : int { WT_F32 = 0, WT_BF16 = 1, WT_FP8 = 2 };
 
@@ -44,6 +45,20 @@ DEC_HD constexpr int gemv_rows_per_thread(int kcb) {
   if (32768 / (G * kcb) < r) r = 32768 / (G * kcb);
   return r < 1 ? 1 : r;
 }
+// Tensor-core operand layouts of MLA attention (bf16, no swizzle).  A core
+// matrix is 8 rows x 8 elements, each row 16 contiguous bytes, 128 bytes in
+// all.  Latent cache of a layer: blocks of kMlaBlock positions; inside a block
+// the core matrix (dims 8k..8k+7, positions 8i..8i+7) sits at k * 1024 + i * 128,
+// so a block is [dim group][position group][8 positions][8 dims] and the
+// (kv_lora + qk_rope) dims of a position are spread over the block.  Absorbed
+// query: the core matrix (dims 8k.., heads 8i..) at k * 2048 + i * 128.
+DEC_HD constexpr long long mla_cache_off(int p_in_block, int d) {  // bytes inside a block
+  return (long long)(d >> 3) * 1024 + (p_in_block >> 3) * 128 + (p_in_block & 7) * 16 + (d & 7) * 2;
+}
+DEC_HD constexpr long long mla_q_off(int h, int d) {  // bytes
+  return (long long)(d >> 3) * 2048 + (h >> 3) * 128 + (h & 7) * 16 + (d & 7) * 2;
+}
+
 enum OpKind : int { OP_GEMV = 0, OP_ATTN = 1, OP_MLA = 2, OP_FINAL = 3 };
 enum Pro : int {
   PRO_NONE = 0,
@@ -83,6 +98,7 @@ struct alignas(16) OpDesc {
   int nsegs;
   Seg seg[kMaxSegs];
   int rows_per_group;  // grouped GEMV: input group = row / rows_per_group (0: one input for all rows)
+  void* qc;            // MLA: absorbed bf16 query in the tensor-core layout (written by absorb_q, read by attention)
   float* out;          // fp32 partial outputs [S][out_stride]
   int out_stride;
   unsigned long long* best;  // LM head: best packed (value, index) key per task, else null
@@ -117,8 +133,8 @@ struct alignas(16) OpDesc {
   PSet ckv;       // MLA: kv_a output (latent then RoPE key)
   const float* kvnorm_g;
   int hq, hkv, hd, gs;
-  int H, HG, kvl, rdim, nope;
-  void* kcache;   // dense: K of this layer [hkv][max_seq][hd]; MLA: [max_seq][kvl + rdim]
+  int H, kvl, rdim, nope;
+  void* kcache;   // dense: K of this layer [hkv][max_seq][hd]; MLA: blocked latent cache (mla_cache_off)
   void* vcache;   // dense: V of this layer
   int cache_bf16;
   int max_seq;

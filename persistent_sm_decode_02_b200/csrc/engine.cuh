@@ -39,6 +39,10 @@ struct Misc {
   uint64_t empty[kStages];
   uint64_t sig_done[kMail];  // consumers -> signaller: task in mailbox slot finished (8 warp arrivals)
   uint64_t sig_free[kMail];  // signaller -> consumers: mailbox slot published and free again
+  uint64_t mma_bar;          // tensor-core MMAs of the current MLA task completed (tcgen05.commit)
+  uint64_t fin_bar;          // every MMA completed before TMEM is freed
+  uint32_t tmem;             // TMEM base address (MLA engine instances)
+  int prod_dep_op;           // op whose producer dependency the producer already waited for
   StepState st;
   volatile int abort;
   int x_op, x_group;     // identity of the input vector currently in the work area
@@ -288,21 +292,21 @@ constexpr int kSrcBatch = 2;                    // residual sources loaded toget
 // the chunks with data (l_c > 0), M = max m_c.  One warp; stores nch weights.
 __device__ __forceinline__ void combine_weights(const float* am, const float* al, int nch, float* w) {
   const int lane = threadIdx.x & 31;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  if (lane < nch) {
-    l0 = ldcg(al + lane);
-    m0 = ldcg(am + lane);
+  float M = -INFINITY;
+  for (int c = lane; c < nch; c += 32)
+    if (ldcg(al + c) > 0.f) M = fmaxf(M, ldcg(am + c));
+  M = warp_max(M);
+  float den = 0.f;
+  for (int c = lane; c < nch; c += 32) {
+    const float l = ldcg(al + c);
+    const float e = l > 0.f ? expf(ldcg(am + c) - M) : 0.f;  // empty chunks (l = 0) get weight 0
+    den += e * l;
+    w[c] = e;
   }
-  if (lane + 32 < nch) {
-    l1 = ldcg(al + lane + 32);
-    m1 = ldcg(am + lane + 32);
-  }
-  const float M = warp_max(fmaxf(l0 > 0.f ? m0 : -INFINITY, l1 > 0.f ? m1 : -INFINITY));
-  const float e0 = l0 > 0.f ? expf(m0 - M) : 0.f, e1 = l1 > 0.f ? expf(m1 - M) : 0.f;
-  const float den = warp_sum(e0 * l0 + e1 * l1);
+  den = warp_sum(den);
   const float inv = den > 0.f ? 1.0f / den : 0.f;
-  if (lane < nch) w[lane] = e0 * inv;
-  if (lane + 32 < nch) w[lane + 32] = e1 * inv;
+  __syncwarp();
+  for (int c = lane; c < nch; c += 32) w[c] *= inv;
 }
 
 // Build the input vector of (op, group) in the work area, all 256 consumer threads.
@@ -467,7 +471,9 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         const float* src = od.ao + ((size_t)(h0 + h) * od.nch) * hd + d;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         int c = 0;
-        for (; c + 4 <= od.nch; c += 4) {
+        // MLA blocks past position pos hold no partials
+        const int nc = mla ? min(od.nch, m->st.pos / kMlaBlock + 1) : od.nch;
+        for (; c + 4 <= nc; c += 4) {
           const float4 a0 = ldcg4(src + (size_t)c * hd), a1 = ldcg4(src + (size_t)(c + 1) * hd);
           const float4 a2 = ldcg4(src + (size_t)(c + 2) * hd), a3 = ldcg4(src + (size_t)(c + 3) * hd);
           fma4(acc, w[c], a0);
@@ -475,7 +481,7 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
           fma4(acc, w[c + 2], a2);
           fma4(acc, w[c + 3], a3);
         }
-        for (; c < od.nch; ++c) fma4(acc, w[c], ldcg4(src + (size_t)c * hd));
+        for (; c < nc; ++c) fma4(acc, w[c], ldcg4(src + (size_t)c * hd));
         store_x4(x, bf, e, acc);
       }
       break;
@@ -644,7 +650,12 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
 #pragma unroll
       for (int i = 0; i < RPT; ++i) {
         const int row = geo.rt * R + rg + G * i;
-        if (row < sg.N) out[row] = acc[i];
+        if (row < sg.N) {
+          out[row] = acc[i];
+          if (od.qc)
+            reinterpret_cast<__nv_bfloat16*>(od.qc)[mla_q_off(row / od.rows_per_group, row % od.rows_per_group) / 2] =
+                __float2bfloat16_rn(acc[i]);
+        }
       }
     }
     return;
@@ -664,6 +675,9 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
     const int row = geo.rt * R + tid;
     if (row < sg.N) {
       od.out[(size_t)geo.s * od.out_stride + sg.out_off + row] = y;
+      if (od.qc)
+        reinterpret_cast<__nv_bfloat16*>(od.qc)[mla_q_off(row / od.rows_per_group, row % od.rows_per_group) / 2] =
+            __float2bfloat16_rn(y);
       if (od.best) key = argmax_key(y, sg.out_off + row);
     }
   }
@@ -704,6 +718,22 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
     case 128: gemv_task<WT, 128>(P, od, op, t, S, g, geo); break;
     case 64: gemv_task<WT, 64>(P, od, op, t, S, g, geo); break;
     default: gemv_task<WT, 32>(P, od, op, t, S, g, geo); break;
+  }
+  if (od.qc) {
+    // absorb_q also feeds the tensor-core MLA attention: gemv_task stored q_lat
+    // rows in bf16; the first tile of head h adds its RoPE'd q_pe (bf16).
+    if (geo.s == 0 && (geo.rt * od.R) % od.rows_per_group == 0) {
+      const int h = geo.rt * od.R / od.rows_per_group, rd = od.rdim, kvl = od.rows_per_group;
+      const int pos = m->st.pos;
+      __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(od.qc);
+      for (int j = threadIdx.x; j < rd / 2; j += kConsumers) {
+        const float a = pset(od.src, h * od.gstride + od.nope + j), b = pset(od.src, h * od.gstride + od.nope + j + rd / 2);
+        const float cs = od.rope_cos[(size_t)pos * (rd / 2) + j], sn = od.rope_sin[(size_t)pos * (rd / 2) + j];
+        q[mla_q_off(h, kvl + j) / 2] = __float2bfloat16_rn(a * cs - b * sn);
+        q[mla_q_off(h, kvl + j + rd / 2) / 2] = __float2bfloat16_rn(a * sn + b * cs);
+      }
+    }
+    fence_async_global();  // read by bulk copies of other CTAs after the op's counter
   }
 }
 
@@ -873,49 +903,48 @@ __device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od,
   }
 }
 
-// MLA absorbed-latent attention (CUDA cores): task = (head group of HG heads, chunk c).
-// s_h(t) = (q_lat^h . c_t + q_pe^h . kpe_t) * scale over the cached rows
-// [c_t | kpe_t]; the chunk holding position pos also normalises, RoPEs and
-// appends the new latent row (RMSNorm of the kv_a latent part, RoPE of its key part).
-__device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
+// MLA absorbed-latent attention on the tensor cores (tcgen05): task c = cache
+// block c (positions [64c, 64c + 64) clipped to 0..pos) for all heads at once,
+// the heads being the MMA's M = 128 rows (DeepSeek-V3 absorbed form, the
+// "MLA" model structure of the pages).
+//   S = Q . C^T : Q = [q_lat | q_pe] bf16 [128 x (kvl + rdim)], C = the block's
+//                 cache rows [64 x (kvl + rdim)]; nine 64-dim K-chunks, each
+//                 ring stage carrying Q's chunk (16 KB) and C's chunk (8 KB).
+//   P = exp(S * scale - m) per head (one thread per head reads its TMEM row),
+//       split into bf16 hi + lo parts so that P keeps ~16 mantissa bits.
+//   O = P . C_lat : two ring stages of 256 latent dims (32 KB each); C is
+//                 read MN-major from the same bytes the S step read K-major.
+// The task publishes (m, l, O) for the split-KV log-sum-exp combine in the uv
+// projection's prologue.  The block holding position pos also normalises and
+// RoPEs the step's new latent row, stores it in the cache and patches it into
+// each stage before the MMAs read the stage.
+// TMEM: 512 fp32 columns x 128 lanes; S uses columns 0..63 and is read out
+// before O (columns 0..511) overwrites it.
+__device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g,
+                                            uint32_t& nmma) {
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nch = od.nch, np = od.np;
-  const int hg = t / nch, c = t % nch;
-  const int HG = od.HG, kvl = od.kvl, rd = od.rdim, rowe = kvl + rd, rowb = rowe * 2, H = od.H;
-  const float scale = od.attn_scale;
-  const int pos = m->st.pos;
-  const ChunkB b = chunk_bounds(c, nch, pos);
-  float* ql = reinterpret_cast<float*>(S.work);            // [HG][kvl]
-  float* qp = ql + HG * kvl;                                // [HG][rd]
-  __nv_bfloat16* newrow = reinterpret_cast<__nv_bfloat16*>(qp + HG * rd);  // [rowe]
-  float* sc = reinterpret_cast<float*>(newrow + rowe);      // [HG][np]
-  const float* cosr = od.rope_cos + (size_t)pos * (rd / 2);
-  const float* sinr = od.rope_sin + (size_t)pos * (rd / 2);
-  const int h0 = hg * HG;
-  // absorbed queries (rounded to bf16), 16-byte loads
-  for (int e = 4 * tid; e < HG * kvl; e += 4 * kConsumers) {
-    const int i = e / kvl, j = e % kvl;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (h0 + i < H) v = pset4(od.qlat, (h0 + i) * kvl + j);
-    v.x = bf16_round(v.x);
-    v.y = bf16_round(v.y);
-    v.z = bf16_round(v.z);
-    v.w = bf16_round(v.w);
-    *reinterpret_cast<float4*>(ql + e) = v;
-  }
-  const int qstride = od.nope + rd;
-  for (int e = tid; e < HG * (rd / 2); e += kConsumers) {
-    const int i = e / (rd / 2), j = e % (rd / 2);
-    float a = 0.f, bb = 0.f;
-    if (h0 + i < H) {
-      a = pset(od.qkv, (h0 + i) * qstride + od.nope + j);
-      bb = pset(od.qkv, (h0 + i) * qstride + od.nope + j + rd / 2);
+  const int pos = m->st.pos, T = pos + 1, nch = od.nch, H = od.H;
+  const int c = t, t0 = c * kMlaBlock;
+  if (t0 >= T) {  // block beyond the sequence: empty partial (l = 0)
+    for (int h = tid; h < H; h += kConsumers) {
+      od.m_out[(size_t)h * nch + c] = -INFINITY;
+      od.l_out[(size_t)h * nch + c] = 0.f;
     }
-    qp[i * rd + j] = bf16_round(a * cosr[j] - bb * sinr[j]);
-    qp[i * rd + j + rd / 2] = bf16_round(a * sinr[j] + bb * cosr[j]);
+    return;
   }
-  if (b.has_new) {
+  const int n = T - t0 < kMlaBlock ? T - t0 : kMlaBlock;
+  const bool has_new = pos < t0 + kMlaBlock;
+  const int pin = pos - t0;
+  const int kvl = od.kvl, rd = od.rdim, rowe = kvl + rd;
+  uint8_t* Phi = S.work;                                                   // [64 pos] x [128 heads] bf16, A layout
+  uint8_t* Plo = S.work + 16384;
+  __nv_bfloat16* newrow = reinterpret_cast<__nv_bfloat16*>(S.work + 32768);  // [rowe]
+  const long long blk_bytes = (long long)rowe * kMlaBlock * 2;
+  uint8_t* blk = reinterpret_cast<uint8_t*>(od.kcache) + (size_t)c * blk_bytes;
+  if (has_new) {
+    const float* cosr = od.rope_cos + (size_t)pos * (rd / 2);
+    const float* sinr = od.rope_sin + (size_t)pos * (rd / 2);
     float ss = 0.f;
     for (int j = tid; j < kvl; j += kConsumers) {
       const float v = pset(od.ckv, j);
@@ -923,125 +952,146 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     }
     const float tot = consumer_sum(ss, m);
     const float inv = 1.0f / sqrtf(tot / (float)kvl + od.eps);
-    __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(od.kcache) + (size_t)pos * rowe;
-    for (int j = tid; j < kvl; j += kConsumers) {
-      const __nv_bfloat16 v = __float2bfloat16_rn(pset(od.ckv, j) * inv * od.kvnorm_g[j]);
-      newrow[j] = v;
-      if (hg == 0) crow[j] = v;
-    }
+    for (int j = tid; j < kvl; j += kConsumers) newrow[j] = __float2bfloat16_rn(pset(od.ckv, j) * inv * od.kvnorm_g[j]);
     for (int j = tid; j < rd / 2; j += kConsumers) {
-      const float a = pset(od.ckv, kvl + j), bb = pset(od.ckv, kvl + j + rd / 2);
-      const __nv_bfloat16 v0 = __float2bfloat16_rn(a * cosr[j] - bb * sinr[j]);
-      const __nv_bfloat16 v1 = __float2bfloat16_rn(a * sinr[j] + bb * cosr[j]);
-      newrow[kvl + j] = v0;
-      newrow[kvl + j + rd / 2] = v1;
-      if (hg == 0) {
-        crow[kvl + j] = v0;
-        crow[kvl + j + rd / 2] = v1;
-      }
+      const float a = pset(od.ckv, kvl + j), b = pset(od.ckv, kvl + j + rd / 2);
+      newrow[kvl + j] = __float2bfloat16_rn(a * cosr[j] - b * sinr[j]);
+      newrow[kvl + j + rd / 2] = __float2bfloat16_rn(a * sinr[j] + b * cosr[j]);
     }
+    named_bar_sync(1, kConsumers);
+    // append to the cache (read by later steps only)
+    for (int k = tid; k < rowe / 8; k += kConsumers)
+      *reinterpret_cast<uint4*>(blk + mla_cache_off(pin, 8 * k)) = reinterpret_cast<const uint4*>(newrow)[k];
   }
-  named_bar_sync(1, kConsumers);
-  // warp w owns heads w*hpw .. ; lane owns latent dims [lane*dpl, +dpl)
-  const int hpw = HG / kConsumerWarps;  // heads per warp (2)
-  const int dpl = kvl / 32;             // 16
-  float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
-  float o[2][16];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int d = 0; d < 16; ++d) o[a][d] = 0.f;
-  const int nck = rowb / 16;  // 72
-  const int nql = kvl / 8;    // chunks of the latent part
-  auto block = [&](const uint8_t* rows, int n) {
-    for (int p = tid; p < HG * n; p += kConsumers) {
-      const int i = p / n, tt = p % n;
-      const uint8_t* row = rows + (size_t)tt * rowb;
-      float dot = 0.f;
-      int jj = tt % nck;
-      for (int j = 0; j < nck; ++j) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(row + jj * 16);
-        const float* qq = jj < nql ? ql + i * kvl + jj * 8 : qp + i * rd + (jj - nql) * 8;
-        const float4 q0 = *reinterpret_cast<const float4*>(qq), q1 = *reinterpret_cast<const float4*>(qq + 4);
-        dot = fmaf(bf16lo(kv.x), q0.x, dot);
-        dot = fmaf(bf16hi(kv.x), q0.y, dot);
-        dot = fmaf(bf16lo(kv.y), q0.z, dot);
-        dot = fmaf(bf16hi(kv.y), q0.w, dot);
-        dot = fmaf(bf16lo(kv.z), q1.x, dot);
-        dot = fmaf(bf16hi(kv.z), q1.y, dot);
-        dot = fmaf(bf16lo(kv.w), q1.z, dot);
-        dot = fmaf(bf16hi(kv.w), q1.w, dot);
-        if (++jj == nck) jj = 0;
-      }
-      sc[i * np + tt] = dot * scale;
-    }
-    named_bar_sync(1, kConsumers);
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-      if (a >= hpw) break;
-      float* s = sc + (warp * hpw + a) * np;
-      float mx = -INFINITY;
-      for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, s[tt]);
-      mx = warp_max(mx);
-      const float mnew = fmaxf(mrun[a], mx);
-      const float alpha = expf(mrun[a] - mnew);
-      float ls = 0.f;
-      for (int tt = lane; tt < n; tt += 32) {
-        const float pv = expf(s[tt] - mnew);
-        s[tt] = pv;
-        ls += pv;
-      }
-      ls = warp_sum(ls);
-      __syncwarp();
-      lrun[a] = lrun[a] * alpha + ls;
-      mrun[a] = mnew;
-#pragma unroll
-      for (int d = 0; d < 16; ++d) o[a][d] *= alpha;
-    }
-    for (int tt = 0; tt < n; ++tt) {
-      const uint4* cr = reinterpret_cast<const uint4*>(rows + (size_t)tt * rowb + lane * dpl * 2);
-      const uint4 c0 = cr[0], c1 = cr[1];
-      const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        if (a >= hpw) break;
-        const float pv = sc[(warp * hpw + a) * np + tt];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          o[a][2 * q] = fmaf(pv, bf16lo(cw[q]), o[a][2 * q]);
-          o[a][2 * q + 1] = fmaf(pv, bf16hi(cw[q]), o[a][2 * q + 1]);
-        }
-      }
-    }
-    named_bar_sync(1, kConsumers);
-  };
-  const int nst = (b.tc - b.t0 + np - 1) / np;
-  for (int st = 0; st < nst; ++st) {
+  const uint32_t tm = m->tmem;
+  constexpr uint32_t kIdS = umma_idesc_bf16(128, kMlaBlock, false);
+  constexpr uint32_t kIdO = umma_idesc_bf16(128, 256, true);
+  // ---- S = Q . C^T over (kvl + rd) / 64 stages
+  const int nS = rowe / 64;
+  for (int j = 0; j < nS; ++j) {
     wait_full(P, S, g, op, t);
-    const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    const int a = b.t0 + st * np;
-    const int n = (b.tc - a) < np ? (b.tc - a) : np;
-    block(stage, n);
-    release_stage(S, g);
+    uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
+    if (has_new) {  // the new row's 64 dims of this chunk
+      if (tid < 8)
+        *reinterpret_cast<uint4*>(stage + 16384 + mla_cache_off(pin, 8 * tid)) =
+            reinterpret_cast<const uint4*>(newrow)[8 * j + tid];
+      fence_async_smem();
+      named_bar_sync(1, kConsumers);
+    }
+    if (warp == 0) {
+      if (lane == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int s = 0; s < 4; ++s)  // K = 16 dims = two core matrices per MMA
+          tc_mma(tm, umma_desc(stage + s * 4096, 2048, 128), umma_desc(stage + 16384 + s * 2048, 1024, 128), kIdS,
+                 (j | s) != 0);
+        tc_commit(&m->empty[g % kStages]);  // the stage is free once these MMAs have read it
+      }
+      __syncwarp();
+    } else {
+      release_stage(S, g);
+    }
     ++g;
   }
-  if (b.has_new) block(reinterpret_cast<const uint8_t*>(newrow), 1);
+  if (tid == 0) tc_commit(&m->mma_bar);
+  // ---- softmax: warps 0..3, thread = head (TMEM lane)
+  const int quad = warp & 3;
+  const int h = 32 * quad + lane;
+  if (warp < 4) {
+    mbar_wait(&m->mma_bar, nmma & 1, P, &m->abort, op, t);
+    __syncwarp();
+    tc_fence_after();
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16), r0);
+    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + 32, r1);
+    tmem_wait_ld();
+    const float scale = od.attn_scale;
+    float mx = -INFINITY;
 #pragma unroll
-  for (int a = 0; a < 2; ++a) {
-    if (a >= hpw) break;
-    const int h = h0 + warp * hpw + a;
-    if (h < H) {
-      const size_t pi = (size_t)h * nch + c;
-      if (lane == 0) {
-        od.m_out[pi] = mrun[a];
-        od.l_out[pi] = lrun[a];
+    for (int i = 0; i < 32; ++i) {
+      if (i < n) mx = fmaxf(mx, __uint_as_float(r0[i]) * scale);
+      if (i + 32 < n) mx = fmaxf(mx, __uint_as_float(r1[i]) * scale);
+    }
+    float l = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {  // positions 8q..8q+7
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float p2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int i = 8 * q + 2 * e + u;
+          const float sv = __uint_as_float(i < 32 ? r0[i & 31] : r1[i & 31]) * scale;
+          p2[u] = i < n ? expf(sv - mx) : 0.f;
+          l += p2[u];
+        }
+        const __nv_bfloat162 ph = __floats2bfloat162_rn(p2[0], p2[1]);
+        const float2 phf = __bfloat1622float2(ph);
+        const __nv_bfloat162 pl = __floats2bfloat162_rn(p2[0] - phf.x, p2[1] - phf.y);
+        hi[e] = *reinterpret_cast<const uint32_t*>(&ph);
+        lo[e] = *reinterpret_cast<const uint32_t*>(&pl);
       }
-      float* dst = od.o_out + pi * kvl + lane * dpl;
+      const int off = q * 2048 + (h >> 3) * 128 + (h & 7) * 16;
+      *reinterpret_cast<uint4*>(Phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(Plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    if (h < H) {
+      od.m_out[(size_t)h * nch + c] = mx;
+      od.l_out[(size_t)h * nch + c] = l;
+    }
+    fence_async_smem();
+    tc_fence_before();
+  }
+  named_bar_sync(1, kConsumers);
+  // ---- O = P . C_lat over kvl / 256 stages (hi and lo parts of P)
+  const int nks = (n + 15) / 16;
+  for (int o = 0; o < kvl / 256; ++o) {
+    wait_full(P, S, g, op, t);
+    uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
+    if (has_new) {
+      if (tid < 32)
+        *reinterpret_cast<uint4*>(stage + mla_cache_off(pin, 8 * tid)) = reinterpret_cast<const uint4*>(newrow)[32 * o + tid];
+      fence_async_smem();
+      named_bar_sync(1, kConsumers);
+    }
+    if (warp == 0) {
+      if (lane == 0) {
+        tc_fence_after();
+        for (int s = 0; s < nks; ++s) {  // K = 16 positions
+          const uint64_t b = umma_desc(stage + s * 256, 128, 1024);  // MN-major: K step 128 B, N step 1024 B
+          tc_mma(tm + 256 * o, umma_desc(Phi + s * 4096, 2048, 128), b, kIdO, s != 0);
+          tc_mma(tm + 256 * o, umma_desc(Plo + s * 4096, 2048, 128), b, kIdO, 1);
+        }
+        tc_commit(&m->empty[g % kStages]);
+      }
+      __syncwarp();
+    } else {
+      release_stage(S, g);
+    }
+    ++g;
+  }
+  if (tid == 0) tc_commit(&m->mma_bar);
+  // ---- epilogue: warp w reads lanes 32 (w % 4).. and columns 256 (w / 4)..
+  mbar_wait(&m->mma_bar, (nmma + 1) & 1, P, &m->abort, op, t);
+  __syncwarp();
+  tc_fence_after();
+  const int col0 = 256 * (warp >> 2);
+#pragma unroll 1
+  for (int cc = 0; cc < 8; ++cc) {
+    uint32_t r[32];
+    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + col0 + 32 * cc, r);
+    tmem_wait_ld();
+    if (h < H) {
+      float4* dst = reinterpret_cast<float4*>(od.o_out + ((size_t)h * nch + c) * kvl + col0 + 32 * cc);
 #pragma unroll
-      for (int d = 0; d < 16; d += 4)
-        *reinterpret_cast<float4*>(dst + d) = make_float4(o[a][d], o[a][d + 1], o[a][d + 2], o[a][d + 3]);
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                             __uint_as_float(r[4 * q + 3]));
     }
   }
+  tc_fence_before();
+  nmma += 2;
 }
 
 // Final op: greedy token = argmax over the LM-head tasks' best keys; advance the step state.
@@ -1205,12 +1255,26 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
                    od.np * rowb, pol_kv);
       }
     } else if (od.kind == OP_MLA) {
-      const int c = t % od.nch;
-      const ChunkB b = chunk_bounds(c, od.nch, pos);
-      const int rowb = (od.kvl + od.rdim) * 2;
-      for (int a = b.t0; a < b.tc && ok; a += od.np) {
-        const int n = (b.tc - a) < od.np ? (b.tc - a) : od.np;
-        ok = issue((const uint8_t*)od.kcache + (size_t)a * rowb, n * rowb, nullptr, 0, 0, pol_kv);
+      // block t: nine (Q chunk, C chunk) stages for S, then two C stages for O
+      if (t * kMlaBlock <= pos) {
+        if (m->prod_dep_op != op) {  // the absorbed query is written by the absorb_q op
+          int r = 1;
+          if (lane == 0) {
+            if (P.persistent) r = wait_counter(P, od.pdep, epoch, &m->abort, op, t) ? 1 : 0;
+            fence_async_global();
+          }
+          if (!__shfl_sync(0xffffffffu, r, 0)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) m->prod_dep_op = op;
+          __syncwarp();
+        }
+        const int rowe = od.kvl + od.rdim;
+        const uint8_t* blk = (const uint8_t*)od.kcache + (size_t)t * rowe * kMlaBlock * 2;
+        const uint8_t* q = (const uint8_t*)od.qc;
+        for (int j = 0; j < rowe / 64 && ok; ++j) ok = issue(q + j * 16384, 16384, blk + j * 8192, 8192, 16384, pol_kv);
+        for (int o = 0; o < od.kvl / 256 && ok; ++o) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
       }
     }
   }
@@ -1300,7 +1364,7 @@ __device__ void signal_loop(const KParams& P, const Smem& S) {
 template <int WT, bool MLA>
 __device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
   Misc* m = S.m;
-  uint32_t g = 0, q = 0;
+  uint32_t g = 0, q = 0, nmma = 0;
   TaskIter it;
   it.init(P);
   int op, t, cur = -1;
@@ -1327,7 +1391,7 @@ __device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
       final_consume(P, od, op, t, S);
     } else {
       if constexpr (MLA)
-        mla_consume(P, od, op, t, S, g);
+        mla_consume(P, od, op, t, S, g, nmma);
       else
         attn_consume(P, od, op, t, S, g);
       if (threadIdx.x == 0) m->x_op = -1;
@@ -1353,6 +1417,7 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
     m->x_op = -1;
     m->x_group = -1;
     m->prod_route_op = -1;
+    m->prod_dep_op = -1;
     m->issued = 0;
     m->consumed = 0;
     for (int i = 0; i < kStages; ++i) {
@@ -1363,14 +1428,25 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
       mbar_init(&m->sig_done[i], kConsumerWarps);
       mbar_init(&m->sig_free[i], 1);
     }
+    mbar_init(&m->mma_bar, 1);
+    mbar_init(&m->fin_bar, 1);
     fence_mbar_init();
     if (P.persistent) {
       __threadfence();
       atomicAdd(P.started, 1u);
     }
   }
-  __syncthreads();
   const int warp = threadIdx.x >> 5;
+  if constexpr (MLA) {  // all 512 TMEM columns: one CTA per SM
+    if (warp == 0) {
+      __syncwarp();  // .sync.aligned: the whole warp, converged
+      tmem_alloc(&m->tmem, 512);
+      tmem_relinquish();
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if constexpr (MLA) tc_fence_after();
   if (warp == kProducerWarp)
     producer_loop(P, S);
   else if (warp == kSignalWarp)
@@ -1378,6 +1454,20 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
   else
     consumer_loop<WT, MLA>(P, S);
   __syncthreads();
+  if constexpr (MLA) {
+    // no MMA may still be running when the columns are freed (after a failure mid-task)
+    if (warp == 0) {
+      if (threadIdx.x == 0) {
+        tc_commit(&m->fin_bar);
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&m->fin_bar, 0) && globaltimer() - t0 < 1000000000ull) {
+        }
+      }
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(m->tmem, 512);
+    }
+  }
   // After a failure, let the copies still in flight land before the CTA exits.
   if (threadIdx.x == 0 && m->issued > m->consumed) {
     const uint64_t t0 = globaltimer();
