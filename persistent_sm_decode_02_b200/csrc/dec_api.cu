@@ -437,7 +437,7 @@ static int build_plan(dec_ctx* c) {
         const OpDesc& ro = c->ops[p.router_op];
         o.routed = PSet{fo.out, fo.S, fo.out_stride, 0};
         o.routed_slot_stride = d;
-        o.route_logits = PSet{ro.out, ro.S, ro.out_stride, 0};
+        o.rt_w = ro.rt_w;
         o.n_experts = f.n_experts;
         o.top_k = f.top_k;
         if (f.n_shared > 0) o.add2 = PSet{fo.out, fo.S, fo.out_stride, f.top_k * d};
@@ -659,6 +659,15 @@ static int build_plan(dec_ctx* c) {
       int ro = P.gemv({{wr, -1, 0}}, d, l, false, "router");
       if (ro < 0) return P.rc;
       ffn_resid(c->ops[ro], true);
+      {
+        OpDesc& o = c->ops[ro];
+        o.router = 1;
+        o.n_experts = E;
+        o.top_k = k;
+        if (dalloc(c, &o.rt_ids, (size_t)k * 4) || dalloc(c, &o.rt_w, (size_t)k * 4)) return DEC_ERR_OOM;
+        CK(cudaMemsetAsync(o.rt_ids, 0, (size_t)k * 4, c->stream));
+        CK(cudaMemsetAsync(o.rt_w, 0, (size_t)k * 4, c->stream));
+      }
       Mat* eg = P.new_mat(DEC_W_EXP_GATE, l, eh, d, E, 0);
       Mat* eu = P.new_mat(DEC_W_EXP_UP, l, eh, d, E, 0);
       Mat* sg = nullptr;
@@ -676,13 +685,12 @@ static int build_plan(dec_ctx* c) {
       }
       int egu = P.gemv(segs, d, l, false, "exp_gate|up");
       if (egu < 0) return P.rc;
-      const OpDesc& rop = c->ops[ro];
-      const PSet rlog{rop.out, rop.S, rop.out_stride, 0};
+      int* rids = c->ops[ro].rt_ids;
       {
         OpDesc& o = c->ops[egu];
         ffn_resid(o, false);
         o.pdep = ro;
-        o.route_logits = rlog;
+        o.rt_ids = rids;
         o.n_experts = E;
         o.top_k = k;
       }
@@ -706,7 +714,7 @@ static int build_plan(dec_ctx* c) {
         o.slot_stride = 2 * eh;
         o.dep[0] = egu;
         o.pdep = ro;
-        o.route_logits = rlog;
+        o.rt_ids = rids;
         o.n_experts = E;
         o.top_k = k;
       }
@@ -744,14 +752,22 @@ static int build_plan(dec_ctx* c) {
 }
 
 // ---------------------------------------------------------- task lists
+// Each op's tasks are cut into n_ctas contiguous runs, one per CTA, starting
+// at a CTA that rotates from op to op so that the remainders spread evenly.
+// Contiguous runs keep a CTA on one input group (expert slot, head) so that
+// the prologue building that group's input runs once per CTA, not per task.
 static int assign_tasks(dec_ctx* c) {
   std::vector<std::vector<int2>> lists(c->n_ctas);
+  const int nc = c->n_ctas;
   int rr = 0;
-  for (int op = 0; op < (int)c->ops.size(); ++op)
-    for (int t = 0; t < c->ops[op].ntasks; ++t) {
-      lists[rr].push_back(make_int2(op, t));
-      rr = (rr + 1) % c->n_ctas;
+  for (int op = 0; op < (int)c->ops.size(); ++op) {
+    const long long n = c->ops[op].ntasks;
+    for (int i = 0; i < nc; ++i) {
+      const int b = (rr + i) % nc;
+      for (long long t = i * n / nc; t < (i + 1) * n / nc; ++t) lists[b].push_back(make_int2(op, (int)t));
     }
+    rr = (int)((rr + n) % nc);
+  }
   std::vector<int2> flat;
   c->task_off.assign(c->n_ctas + 1, 0);
   for (int b = 0; b < c->n_ctas; ++b) {
@@ -932,11 +948,15 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
     if ((rc = dalloc(c, &c->d_route_dump, (size_t)c->n_moe * f.top_k * 4))) return rc;
     int i = 0;
     for (auto& o : c->ops)
-      if (o.kind == OP_GEMV && o.pdep >= 0 && o.pro == PRO_RESID_NORM) o.route_dump = c->d_route_dump + f.top_k * i++;
+      if (o.router) o.route_dump = c->d_route_dump + f.top_k * i++;
   }
+  // per op: the dependency counter, then (routers) the finished-task counter
+  if ((rc = dalloc(c, &c->d_counters, c->ops.size() * 8))) return rc;
+  CK(cudaMemsetAsync(c->d_counters, 0, c->ops.size() * 8, c->stream));
+  for (size_t i = 0; i < c->ops.size(); ++i)
+    if (c->ops[i].router) c->ops[i].fin = c->d_counters + c->ops.size() + i;
   if ((rc = upload_ops(c))) return rc;
   if ((rc = assign_tasks(c))) return rc;
-  if ((rc = dalloc(c, &c->d_counters, c->ops.size() * 4))) return rc;
   if ((rc = dalloc(c, &c->d_state, sizeof(StepState)))) return rc;
   if ((rc = dalloc(c, &c->d_started, 4))) return rc;
   if ((rc = dalloc(c, &c->d_status, sizeof(Status)))) return rc;
@@ -990,7 +1010,7 @@ extern "C" int dec_reset(dec_ctx* c) {
   CK(cudaSetDevice(c->cfg.device));
   cudaStreamSynchronize(c->stream);
   (void)cudaGetLastError();
-  CK(cudaMemsetAsync(c->d_counters, 0, c->ops.size() * 4, c->stream));
+  CK(cudaMemsetAsync(c->d_counters, 0, c->ops.size() * 8, c->stream));
   CK(cudaMemsetAsync(c->d_started, 0, 4, c->stream));
   CK(cudaMemsetAsync(c->d_status, 0, sizeof(Status), c->stream));
   StepState st{1, 0, 0, 0};

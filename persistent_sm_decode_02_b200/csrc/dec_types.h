@@ -113,9 +113,12 @@ struct alignas(16) OpDesc {
   PSet add, add2;          // summed with weight 1 (ptr null = unused)
   PSet routed;             // routed expert outputs, slot j at off + j * routed_slot_stride
   int routed_slot_stride;
-  PSet route_logits;       // router logits (E values)
   int n_experts, top_k;
-  int* route_dump;         // routed GEMV ops: the producer stores the chosen expert ids here
+  int router;              // 1: the router GEMV; its last task turns the logits into the top-k
+  unsigned* fin;           // router: tasks finished (cumulative over steps), to find the last one
+  int* rt_ids;             // router: top-k expert ids it writes; routed GEMV ops: ids their producer reads
+  float* rt_w;             // router: renormalised top-k weights it writes; RESID_NORM: weights it reads
+  int* route_dump;         // router: the chosen expert ids are also stored here (debug dump)
   const float* gain;
   float eps;
   float* h_out;            // RESID_NORM: the op's task 0 stores h here

@@ -43,6 +43,7 @@ struct Misc {
   uint64_t fin_bar;          // every MMA completed before TMEM is freed
   uint32_t tmem;             // TMEM base address (MLA engine instances)
   int prod_dep_op;           // op whose producer dependency the producer already waited for
+  int last_task;             // the current router task is the op's last one to finish
   StepState st;
   volatile int abort;
   int x_op, x_group;     // identity of the input vector currently in the work area
@@ -321,7 +322,7 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
     case PRO_NORM_SUM: {
       const bool resid = od.pro == PRO_RESID_NORM;
       if (resid && od.routed.ptr) {
-        if (tid < 32) warp_route(od.route_logits, od.n_experts, od.top_k, nullptr, m->cons_w);
+        if (tid < od.top_k) m->cons_w[tid] = __ldcg(od.rt_w + tid);  // written by the router's last task
         named_bar_sync(1, kConsumers);
       }
       float4 v[kMaxQ];
@@ -719,6 +720,22 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
     case 64: gemv_task<WT, 64>(P, od, op, t, S, g, geo); break;
     default: gemv_task<WT, 32>(P, od, op, t, S, g, geo); break;
   }
+  if (od.router) {
+    // The task that finishes the router op last sums the logits' split-K
+    // partials and stores the top-k ids and weights once for all readers.
+    __threadfence();
+    named_bar_sync(1, kConsumers);
+    if (threadIdx.x == 0) {
+      const unsigned prev = atomicAdd(od.fin, 1u);
+      m->last_task = prev + 1 == (unsigned)m->st.epoch * (unsigned)od.ntasks;
+    }
+    named_bar_sync(1, kConsumers);
+    if (m->last_task && threadIdx.x < 32) {
+      __threadfence();
+      warp_route(PSet{od.out, od.S, od.out_stride, 0}, od.n_experts, od.top_k, od.rt_ids, od.rt_w);
+      if (od.route_dump && threadIdx.x < od.top_k) od.route_dump[threadIdx.x] = __ldcg(od.rt_ids + threadIdx.x);
+    }
+  }
   if (od.qc) {
     // absorb_q also feeds the tensor-core MLA attention: gemv_task stored q_lat
     // rows in bf16; the first tile of head h adds its RoPE'd q_pe (bf16).
@@ -943,20 +960,28 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   const long long blk_bytes = (long long)rowe * kMlaBlock * 2;
   uint8_t* blk = reinterpret_cast<uint8_t*>(od.kcache) + (size_t)c * blk_bytes;
   if (has_new) {
-    const float* cosr = od.rope_cos + (size_t)pos * (rd / 2);
-    const float* sinr = od.rope_sin + (size_t)pos * (rd / 2);
-    float ss = 0.f;
-    for (int j = tid; j < kvl; j += kConsumers) {
-      const float v = pset(od.ckv, j);
-      ss += v * v;
-    }
-    const float tot = consumer_sum(ss, m);
+    // c = bf16(RMSNorm(kv_a latent) * g); k_pe = bf16(RoPE(kv_a rope part)); 16-byte loads of the split partials
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (4 * tid < kvl) v = pset4(od.ckv, 4 * tid);
+    const float tot = consumer_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, m);
     const float inv = 1.0f / sqrtf(tot / (float)kvl + od.eps);
-    for (int j = tid; j < kvl; j += kConsumers) newrow[j] = __float2bfloat16_rn(pset(od.ckv, j) * inv * od.kvnorm_g[j]);
-    for (int j = tid; j < rd / 2; j += kConsumers) {
-      const float a = pset(od.ckv, kvl + j), b = pset(od.ckv, kvl + j + rd / 2);
-      newrow[kvl + j] = __float2bfloat16_rn(a * cosr[j] - b * sinr[j]);
-      newrow[kvl + j + rd / 2] = __float2bfloat16_rn(a * sinr[j] + b * cosr[j]);
+    if (4 * tid < kvl) {
+      const float4 g4 = __ldg(reinterpret_cast<const float4*>(od.kvnorm_g + 4 * tid));
+      reinterpret_cast<__nv_bfloat162*>(newrow)[2 * tid] = __floats2bfloat162_rn(v.x * inv * g4.x, v.y * inv * g4.y);
+      reinterpret_cast<__nv_bfloat162*>(newrow)[2 * tid + 1] = __floats2bfloat162_rn(v.z * inv * g4.z, v.w * inv * g4.w);
+    }
+    const int rq = tid - kvl / 4;  // RoPE: 4 pairs (j, j + rd/2) per thread
+    if (rq >= 0 && 4 * rq < rd / 2) {
+      const int j = 4 * rq;
+      const float4 a = pset4(od.ckv, kvl + j), b = pset4(od.ckv, kvl + j + rd / 2);
+      const float4 cs = __ldg(reinterpret_cast<const float4*>(od.rope_cos + (size_t)pos * (rd / 2) + j));
+      const float4 sn = __ldg(reinterpret_cast<const float4*>(od.rope_sin + (size_t)pos * (rd / 2) + j));
+      __nv_bfloat162* lo = reinterpret_cast<__nv_bfloat162*>(newrow + kvl + j);
+      __nv_bfloat162* hi = reinterpret_cast<__nv_bfloat162*>(newrow + kvl + j + rd / 2);
+      lo[0] = __floats2bfloat162_rn(a.x * cs.x - b.x * sn.x, a.y * cs.y - b.y * sn.y);
+      lo[1] = __floats2bfloat162_rn(a.z * cs.z - b.z * sn.z, a.w * cs.w - b.w * sn.w);
+      hi[0] = __floats2bfloat162_rn(a.x * sn.x + b.x * cs.x, a.y * sn.y + b.y * cs.y);
+      hi[1] = __floats2bfloat162_rn(a.z * sn.z + b.z * cs.z, a.w * sn.w + b.w * cs.w);
     }
     named_bar_sync(1, kConsumers);
     // append to the cache (read by later steps only)
@@ -994,56 +1019,57 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     ++g;
   }
   if (tid == 0) tc_commit(&m->mma_bar);
-  // ---- softmax: warps 0..3, thread = head (TMEM lane)
-  const int quad = warp & 3;
+  // ---- softmax: all 8 warps; warp w reads TMEM lanes 32 (w % 4).. (heads) and
+  // columns 32 (w / 4).. (positions); row max and sum meet in shared memory.
+  const int quad = warp & 3, half = warp >> 2;
   const int h = 32 * quad + lane;
-  if (warp < 4) {
-    mbar_wait(&m->mma_bar, nmma & 1, P, &m->abort, op, t);
-    __syncwarp();
-    tc_fence_after();
-    uint32_t r0[32], r1[32];
-    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16), r0);
-    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + 32, r1);
+  float* red = m->red;  // [2][128]
+  mbar_wait(&m->mma_bar, nmma & 1, P, &m->abort, op, t);
+  __syncwarp();
+  tc_fence_after();
+  {
+    uint32_t r[32];
+    tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + 32 * half, r);
     tmem_wait_ld();
-    const float scale = od.attn_scale;
+    const float sl2 = od.attn_scale * 1.4426950408889634f;  // scale * log2(e): p = 2^(s * sl2 - max)
+    const int nv = n - 32 * half;                             // valid columns of this half
     float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i < n) mx = fmaxf(mx, __uint_as_float(r0[i]) * scale);
-      if (i + 32 < n) mx = fmaxf(mx, __uint_as_float(r1[i]) * scale);
-    }
+    for (int i = 0; i < 32; ++i)
+      if (i < nv) mx = fmaxf(mx, __uint_as_float(r[i]) * sl2);
+    red[128 * half + h] = mx;
+    named_bar_sync(1, kConsumers);
+    mx = fmaxf(red[h], red[128 + h]);  // n >= 1: finite
     float l = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {  // positions 8q..8q+7
+    for (int q = 0; q < 4; ++q) {  // positions 32 half + 8q .. + 7
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float p2[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int i = 8 * q + 2 * e + u;
-          const float sv = __uint_as_float(i < 32 ? r0[i & 31] : r1[i & 31]) * scale;
-          p2[u] = i < n ? expf(sv - mx) : 0.f;
-          l += p2[u];
-        }
-        const __nv_bfloat162 ph = __floats2bfloat162_rn(p2[0], p2[1]);
+        const int i0 = 8 * q + 2 * e;
+        const float p0 = i0 < nv ? ex2_approx(__uint_as_float(r[i0]) * sl2 - mx) : 0.f;
+        const float p1 = i0 + 1 < nv ? ex2_approx(__uint_as_float(r[i0 + 1]) * sl2 - mx) : 0.f;
+        l += p0 + p1;
+        const __nv_bfloat162 ph = __floats2bfloat162_rn(p0, p1);
         const float2 phf = __bfloat1622float2(ph);
-        const __nv_bfloat162 pl = __floats2bfloat162_rn(p2[0] - phf.x, p2[1] - phf.y);
+        const __nv_bfloat162 pl = __floats2bfloat162_rn(p0 - phf.x, p1 - phf.y);
         hi[e] = *reinterpret_cast<const uint32_t*>(&ph);
         lo[e] = *reinterpret_cast<const uint32_t*>(&pl);
       }
-      const int off = q * 2048 + (h >> 3) * 128 + (h & 7) * 16;
+      const int off = (4 * half + q) * 2048 + (h >> 3) * 128 + (h & 7) * 16;
       *reinterpret_cast<uint4*>(Phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(Plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    if (h < H) {
-      od.m_out[(size_t)h * nch + c] = mx;
-      od.l_out[(size_t)h * nch + c] = l;
-    }
+    named_bar_sync(1, kConsumers);  // both halves read red[] before it is reused
+    red[128 * half + h] = l;
     fence_async_smem();
     tc_fence_before();
+    named_bar_sync(1, kConsumers);
+    if (half == 0 && h < H) {  // (m, l) in natural-log units for the combine
+      od.m_out[(size_t)h * nch + c] = mx * 0.6931471805599453f;  // log2 units -> natural log
+      od.l_out[(size_t)h * nch + c] = red[h] + red[128 + h];
+    }
   }
-  named_bar_sync(1, kConsumers);
   // ---- O = P . C_lat over kvl / 256 stages (hi and lo parts of P)
   const int nks = (n + 15) / 16;
   for (int o = 0; o < kvl / 256; ++o) {
@@ -1072,23 +1098,33 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     ++g;
   }
   if (tid == 0) tc_commit(&m->mma_bar);
-  // ---- epilogue: warp w reads lanes 32 (w % 4).. and columns 256 (w / 4)..
+  // ---- epilogue: warp w reads lanes 32 (w % 4).. and columns 256 (w / 4)..; each
+  // 32 x 32 tile goes through shared memory so that the stores are coalesced
   mbar_wait(&m->mma_bar, (nmma + 1) & 1, P, &m->abort, op, t);
   __syncwarp();
   tc_fence_after();
-  const int col0 = 256 * (warp >> 2);
+  const int col0 = 256 * half;
+  float* tile = reinterpret_cast<float*>(S.work) + warp * (32 * 36);  // [32 heads][36] (P and newrow are dead)
 #pragma unroll 1
   for (int cc = 0; cc < 8; ++cc) {
     uint32_t r[32];
     tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + col0 + 32 * cc, r);
     tmem_wait_ld();
-    if (h < H) {
-      float4* dst = reinterpret_cast<float4*>(od.o_out + ((size_t)h * nch + c) * kvl + col0 + 32 * cc);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                             __uint_as_float(r[4 * q + 3]));
+    for (int q = 0; q < 8; ++q)
+      *reinterpret_cast<float4*>(tile + lane * 36 + 4 * q) =
+          make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                      __uint_as_float(r[4 * q + 3]));
+    __syncwarp();
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {  // 4 heads x 32 columns per instruction
+      const int i = 4 * it + (lane >> 3), q = lane & 7;
+      const int hh = 32 * quad + i;
+      if (hh < H)
+        *reinterpret_cast<float4*>(od.o_out + ((size_t)hh * nch + c) * kvl + col0 + 32 * cc + 4 * q) =
+            *reinterpret_cast<const float4*>(tile + i * 36 + 4 * q);
     }
+    __syncwarp();
   }
   tc_fence_before();
   nmma += 2;
@@ -1231,12 +1267,8 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
             ok = false;
             break;
           }
-          warp_route(od.route_logits, od.n_experts, od.top_k, m->prod_idx, nullptr);
-          if (lane == 0) {
-            m->prod_route_op = od.pdep;
-            if (od.route_dump)
-              for (int j = 0; j < od.top_k; ++j) od.route_dump[j] = m->prod_idx[j];
-          }
+          if (lane < od.top_k) m->prod_idx[lane] = __ldcg(od.rt_ids + lane);  // written by the router's last task
+          if (lane == 0) m->prod_route_op = od.pdep;
           __syncwarp();
         }
         base += (size_t)m->prod_idx[sg.slot] * sg.w_estride;

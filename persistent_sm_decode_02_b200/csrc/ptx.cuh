@@ -118,6 +118,13 @@ __device__ __forceinline__ __half2 e4m3x2_to_half2(uint16_t v) {
   return *reinterpret_cast<__half2*>(&r);
 }
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx; relative error ~2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
