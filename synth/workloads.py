@@ -55,6 +55,12 @@ WORKLOADS = {
     "moe_mla_fp8_8k": dict(_BASE_MLA, n_layers=12, d_model=7168, n_heads=128, q_lora=1536, n_dense_layers=3,
                            ffn_hidden=18432, n_experts=256, top_k=8, expert_hidden=2048, vocab=129280,
                            weight_dtype="fp8", ctx=8192, n_decode=1024, seed=1004, cache_from="synthetic"),
+    # --- profiling case: one MoE layer of the full-size MLA model with 16 experts and a
+    # short vocabulary (~1.1 GB of weights, ~0.7 GB streamed per step: above the L2, small
+    # enough for an ncu capture that saves and restores device memory between passes)
+    "prof_mla_moe_fp8": dict(_BASE_MLA, n_layers=1, d_model=7168, n_heads=128, q_lora=1536, n_dense_layers=0,
+                             ffn_hidden=18432, n_experts=16, top_k=8, expert_hidden=2048, vocab=8192,
+                             weight_dtype="fp8", ctx=1024, n_decode=64, seed=3004, cache_from="synthetic"),
     # --- small parity cases (several tiles, ragged tails, all code paths)
     "small_dense_bf16": dict(_BASE_DENSE, n_layers=2, d_model=384, n_heads=6, n_kv_heads=2, head_dim=64,
                              ffn_hidden=1000, vocab=1000, weight_dtype="bf16", ctx=77, n_decode=6, seed=2002,
