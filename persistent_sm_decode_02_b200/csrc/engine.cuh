@@ -326,6 +326,16 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         named_bar_sync(1, kConsumers);
       }
       float4 v[kMaxQ];
+      // The gains (often read from HBM) are copied asynchronously into the work area
+      // behind the input vector, so their latency overlaps the base and source loads;
+      // each thread later reads back only the chunks it copied itself.
+      const int goff = ((od.Kpad * (bf ? 2 : 4)) + 15) & ~15;
+      float* gs = reinterpret_cast<float*>(S.work + goff);
+      const bool stage_g = goff + 4 * n <= kWorkBytes;
+      if (stage_g) {
+        for (int e = 4 * tid; e < n; e += 4 * kConsumers) cp_async16(gs + e, od.gain + e);
+        cp_async_commit();
+      }
       // base
 #pragma unroll
       for (int i = 0; i < kMaxQ; ++i) {
@@ -389,13 +399,15 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
       float ss = 0.f;
 #pragma unroll
       for (int i = 0; i < kMaxQ; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+      if (stage_g) cp_async_wait_all();
       const float tot = consumer_sum(ss, m);
       const float inv = 1.0f / sqrtf(tot / (float)n + od.eps);
 #pragma unroll
       for (int i = 0; i < kMaxQ; ++i) {
         const int e = 4 * (tid + i * kConsumers);
         if (e < n) {
-          const float4 g = __ldg(reinterpret_cast<const float4*>(od.gain + e));
+          const float4 g = stage_g ? *reinterpret_cast<const float4*>(gs + e)
+                                   : __ldg(reinterpret_cast<const float4*>(od.gain + e));
           float4 y;
           y.x = v[i].x * inv * g.x;
           y.y = v[i].y * inv * g.y;

@@ -107,6 +107,14 @@ __device__ __forceinline__ int named_bar_or(int id, int n, int pred) {
   return r;
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only), its commit and the
+// thread's wait for all of its committed copies.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // L2-coherent loads of data written by other CTAs during the same launch.
 __device__ __forceinline__ float ldcg(const float* p) { return __ldcg(p); }
 
