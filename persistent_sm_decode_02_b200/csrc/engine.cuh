@@ -783,23 +783,94 @@ __device__ __forceinline__ ChunkB chunk_bounds(int c, int nch, int pos) {
   return b;
 }
 
-// Dense GQA split-KV attention: task = (kv head g, chunk c); all gs query heads of g.
-// Each head keeps a running (max m, sum l, weighted values o) over the chunk
-// (online softmax, Milakov & Gimelshein 2018) and publishes them for the
-// log-sum-exp combine in the output projection's prologue.
-__device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
+// Dense GQA split-KV attention: task = (kv head, position chunk c), all gs query heads of
+// the kv head (GQA: query head i reads kv head i * hkv / hq).  Each head keeps a running
+// (max m, sum l, weighted values o) over the chunk (online softmax, Milakov & Gimelshein
+// 2018) and publishes them for the log-sum-exp combine in the output projection's prologue.
+// Work split, so that the chunk streams at the ring's rate on CUDA cores: warp w takes
+// positions w, w + 8, ... of every ring stage; lane l holds dims [dpl l, dpl l + dpl) of
+// the G (gs rounded up to a power of two) query heads.  Per position the G partial dot
+// products are reduced over the warp by one multi-value butterfly (after it, lane l holds
+// the full score of one head), the G scores are broadcast, and every lane updates its
+// warp's state with base-2 exponentials.  The 8 warps' states merge once per task.
+template <int G>
+__device__ __forceinline__ float group_reduce(float (&v)[G], int lane) {
+#pragma unroll
+  for (int cnt = G, b = 16; cnt > 1; cnt >>= 1, b >>= 1) {
+    const bool up = (lane & b) != 0;
+#pragma unroll
+    for (int i = 0; i < cnt / 2; ++i) {
+      const float send = up ? v[i] : v[i + cnt / 2];
+      const float keep = up ? v[i + cnt / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, b);
+    }
+  }
+  constexpr int kLog = G >= 8 ? 3 : G >= 4 ? 2 : G >= 2 ? 1 : 0;
+#pragma unroll
+  for (int b = 16 >> kLog; b >= 1; b >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], b);
+  return v[0];
+}
+
+// Lane that holds head h's score after group_reduce<G>.
+template <int G>
+__device__ __forceinline__ int group_holder(int h) {
+  constexpr int kLog = G >= 8 ? 3 : G >= 4 ? 2 : G >= 2 ? 1 : 0;
+  int lane = 0;
+#pragma unroll
+  for (int k = 0; k < kLog; ++k) lane |= ((h >> (kLog - 1 - k)) & 1) << (4 - k);
+  return lane;
+}
+
+template <int DPL>
+__device__ __forceinline__ void load_dims(const uint8_t* row, int cbf, int lane, float (&x)[DPL]) {
+  if (cbf) {
+    if constexpr (DPL == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(row + lane * 8);
+      x[0] = bf16lo(u.x);
+      x[1] = bf16hi(u.x);
+      x[2] = bf16lo(u.y);
+      x[3] = bf16hi(u.y);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+      x[0] = bf16lo(u);
+      x[1] = bf16hi(u);
+    }
+  } else {
+    if constexpr (DPL == 4) {
+      const float4 f = *reinterpret_cast<const float4*>(row + lane * 16);
+      x[0] = f.x;
+      x[1] = f.y;
+      x[2] = f.z;
+      x[3] = f.w;
+    } else {
+      const float2 f = *reinterpret_cast<const float2*>(row + lane * 8);
+      x[0] = f.x;
+      x[1] = f.y;
+    }
+  }
+}
+
+// G: query heads of the kv head rounded up to a power of two; DPL = head_dim / 32.
+// A warp carries at most 4 heads: for G = 8 the warps form two sets of 4 (heads 0-3 and
+// 4-7), each set taking every 4th position.
+template <int G, int DPL>
+__device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
+                                          uint32_t& g) {
+  constexpr int HW = G < 4 ? G : 4;        // heads per warp
+  constexpr int SETS = G / HW;             // warp sets (1 or 2)
+  constexpr int WPS = kConsumerWarps / SETS;  // warps per set
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int set = warp / WPS, wi = warp % WPS;
   const int nch = od.nch, np = od.np;
   const int kvh = t / nch, c = t % nch;
   const int pos = m->st.pos;
   const ChunkB b = chunk_bounds(c, nch, pos);
   const int hd = od.hd, gs = od.gs, cbf = od.cache_bf16, cb = cbf ? 2 : 4;
   const int rowb = hd * cb;
-  const float scale = od.attn_scale;
-  float* q_s = reinterpret_cast<float*>(S.work);           // [gs][hd]
-  uint8_t* new_s = S.work + gs * hd * 4;                    // K row then V row (cache dtype)
-  float* sc = reinterpret_cast<float*>(new_s + 2 * rowb);   // [gs][np]
+  float* q_s = reinterpret_cast<float*>(S.work);                   // [gs][hd]
+  uint8_t* new_s = S.work + gs * hd * 4;                            // K row then V row (cache dtype)
+  float* mg = reinterpret_cast<float*>(S.work + 8192);             // merge area: [8 warps][HW][hd + 2]
   const int half = hd / 2;
   const float* cosr = od.rope_cos + (size_t)pos * (od.rope_dim / 2);
   const float* sinr = od.rope_sin + (size_t)pos * (od.rope_dim / 2);
@@ -842,73 +913,42 @@ __device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od,
     }
   }
   named_bar_sync(1, kConsumers);
-  // per-head running state: warp i < gs owns head i; lane owns hd/32 dims
-  const int dpl = hd / 32;
-  float mrun = -INFINITY, lrun = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
-  const int nck = rowb / 16;
-  auto block = [&](const uint8_t* Kp, const uint8_t* Vp, int n) {
-    for (int p = tid; p < gs * n; p += kConsumers) {
-      const int i = p / n, tt = p % n;
-      const float* q = q_s + i * hd;
-      const uint8_t* krow = Kp + (size_t)tt * rowb;
-      float dot = 0.f;
-      int jj = tt % nck;
-      for (int j = 0; j < nck; ++j) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(krow + jj * 16);
-        if (cbf) {
-          const float4 q0 = *reinterpret_cast<const float4*>(q + jj * 8);
-          const float4 q1 = *reinterpret_cast<const float4*>(q + jj * 8 + 4);
-          dot = fmaf(bf16lo(kv.x), q0.x, dot);
-          dot = fmaf(bf16hi(kv.x), q0.y, dot);
-          dot = fmaf(bf16lo(kv.y), q0.z, dot);
-          dot = fmaf(bf16hi(kv.y), q0.w, dot);
-          dot = fmaf(bf16lo(kv.z), q1.x, dot);
-          dot = fmaf(bf16hi(kv.z), q1.y, dot);
-          dot = fmaf(bf16lo(kv.w), q1.z, dot);
-          dot = fmaf(bf16hi(kv.w), q1.w, dot);
-        } else {
-          const float4 q0 = *reinterpret_cast<const float4*>(q + jj * 4);
-          dot = fmaf(__uint_as_float(kv.x), q0.x, dot);
-          dot = fmaf(__uint_as_float(kv.y), q0.y, dot);
-          dot = fmaf(__uint_as_float(kv.z), q0.z, dot);
-          dot = fmaf(__uint_as_float(kv.w), q0.w, dot);
-        }
-        if (++jj == nck) jj = 0;
-      }
-      sc[i * np + tt] = dot * scale;
+  // this lane's dims of the warp's heads (heads past gs are zero)
+  float q[HW][DPL], o[HW][DPL], mr[HW], lr[HW];
+#pragma unroll
+  for (int h = 0; h < HW; ++h) {
+    const int qh = set * HW + h;
+    mr[h] = -INFINITY;
+    lr[h] = 0.f;
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) {
+      q[h][d] = qh < gs ? q_s[qh * hd + lane * DPL + d] : 0.f;
+      o[h][d] = 0.f;
     }
-    named_bar_sync(1, kConsumers);
-    if (warp < gs) {
-      float* s = sc + warp * np;
-      float mx = -INFINITY;
-      for (int tt = lane; tt < n; tt += 32) mx = fmaxf(mx, s[tt]);
-      mx = warp_max(mx);
-      const float mnew = fmaxf(mrun, mx);
-      const float alpha = expf(mrun - mnew);
-      float ls = 0.f;
-      for (int tt = lane; tt < n; tt += 32) {
-        const float pv = expf(s[tt] - mnew);
-        s[tt] = pv;
-        ls += pv;
-      }
-      ls = warp_sum(ls);
-      __syncwarp();
-      lrun = lrun * alpha + ls;
-      mrun = mnew;
-      for (int d = 0; d < dpl; ++d) o[d] *= alpha;
-      for (int tt = 0; tt < n; ++tt) {
-        const float pv = s[tt];
-        const uint8_t* vrow = Vp + (size_t)tt * rowb;
-        if (cbf) {
-          const __nv_bfloat16* vv = reinterpret_cast<const __nv_bfloat16*>(vrow) + lane * dpl;
-          for (int d = 0; d < dpl; ++d) o[d] = fmaf(pv, __bfloat162float(vv[d]), o[d]);
-        } else {
-          const float* vv = reinterpret_cast<const float*>(vrow) + lane * dpl;
-          for (int d = 0; d < dpl; ++d) o[d] = fmaf(pv, vv[d], o[d]);
-        }
-      }
+  }
+  const float sl2 = od.attn_scale * 1.4426950408889634f;  // scores in base-2 units
+  auto position = [&](const uint8_t* krow, const uint8_t* vrow) {
+    float kf[DPL], vf[DPL], v[HW];
+    load_dims<DPL>(krow, cbf, lane, kf);
+    load_dims<DPL>(vrow, cbf, lane, vf);
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+      float x = 0.f;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) x = fmaf(q[h][d], kf[d], x);
+      v[h] = x;
     }
-    named_bar_sync(1, kConsumers);
+    const float mine = group_reduce<HW>(v, lane);
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+      const float s = __shfl_sync(0xffffffffu, mine, group_holder<HW>(h)) * sl2;
+      const float mn = fmaxf(mr[h], s);
+      const float corr = ex2_approx(mr[h] - mn), p = ex2_approx(s - mn);
+      lr[h] = lr[h] * corr + p;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) o[h][d] = fmaf(p, vf[d], o[h][d] * corr);
+      mr[h] = mn;
+    }
   };
   const int nst = (b.tc - b.t0 + np - 1) / np;
   for (int st = 0; st < nst; ++st) {
@@ -916,20 +956,66 @@ __device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od,
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
     const int a = b.t0 + st * np;
     const int n = (b.tc - a) < np ? (b.tc - a) : np;
-    block(stage, stage + (size_t)np * rowb, n);
+    for (int tt = wi; tt < n; tt += WPS) position(stage + (size_t)tt * rowb, stage + (size_t)(np + tt) * rowb);
     release_stage(S, g);
     ++g;
   }
-  if (b.has_new) block(new_s, new_s + rowb, 1);
-  if (warp < gs) {
-    const int qh = kvh * gs + warp;
-    const size_t pi = (size_t)qh * nch + c;
+  if (b.has_new && wi == 0) position(new_s, new_s + rowb);
+  // merge the warps of each head's set: M = max m_w, o = sum 2^(m_w - M) o_w, l = sum 2^(m_w - M) l_w
+  const int stride = hd + 2;
+#pragma unroll
+  for (int h = 0; h < HW; ++h) {
+    float* rec = mg + (warp * HW + h) * stride;
     if (lane == 0) {
-      od.m_out[pi] = mrun;
-      od.l_out[pi] = lrun;
+      rec[hd] = mr[h];
+      rec[hd + 1] = lr[h];
     }
-    for (int d = 0; d < dpl; ++d) od.o_out[pi * hd + lane * dpl + d] = o[d];
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) rec[lane * DPL + d] = o[h][d];
   }
+  named_bar_sync(1, kConsumers);
+  for (int e = tid; e < gs * hd; e += kConsumers) {
+    const int qh = e / hd, d = e % hd;
+    const int st2 = qh / HW, h = qh % HW;
+    float M = -INFINITY;
+    for (int w = st2 * WPS; w < (st2 + 1) * WPS; ++w) M = fmaxf(M, mg[(w * HW + h) * stride + hd]);
+    float acc = 0.f, l = 0.f;
+    if (M != -INFINITY)
+      for (int w = st2 * WPS; w < (st2 + 1) * WPS; ++w) {
+        const float* rec = mg + (w * HW + h) * stride;
+        const float f = ex2_approx(rec[hd] - M);
+        acc = fmaf(f, rec[d], acc);
+        l = fmaf(f, rec[hd + 1], l);
+      }
+    const size_t pi = (size_t)(kvh * gs + qh) * nch + c;
+    od.o_out[pi * hd + d] = acc;
+    if (d == 0) {
+      od.m_out[pi] = M == -INFINITY ? -INFINITY : M * 0.6931471805599453f;  // base 2 -> natural log
+      od.l_out[pi] = l;
+    }
+  }
+  named_bar_sync(1, kConsumers);  // the merge area is free again
+}
+
+template <int DPL>
+__device__ __forceinline__ void attn_consume_dpl(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
+                                                 uint32_t& g) {
+  const int gs = od.gs;
+  if (gs <= 1)
+    attn_task<1, DPL>(P, od, op, t, S, g);
+  else if (gs <= 2)
+    attn_task<2, DPL>(P, od, op, t, S, g);
+  else if (gs <= 4)
+    attn_task<4, DPL>(P, od, op, t, S, g);
+  else
+    attn_task<8, DPL>(P, od, op, t, S, g);
+}
+
+__device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g) {
+  if (od.hd == 128)
+    attn_consume_dpl<4>(P, od, op, t, S, g);
+  else
+    attn_consume_dpl<2>(P, od, op, t, S, g);
 }
 
 // MLA absorbed-latent attention on the tensor cores (tcgen05): task c = cache
