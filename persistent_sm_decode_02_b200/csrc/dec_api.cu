@@ -83,7 +83,10 @@ Geo gemv_geometry(int K, int wb) {
   return g;
 }
 
-int choose_split(int ntiles, int nst_total, int n_ctas, bool force_one) {
+// Split-K factor S of a GEMV op, in units of ring stages on the busiest CTA: its tasks'
+// stages plus a fixed cost per task, plus the consumer's prologue, which reads all S
+// partial vectors (out_rows fp32 values each) on every CTA.
+int choose_split(int ntiles, int nst_total, int n_ctas, long long out_rows, bool force_one) {
   if (force_one) return 1;
   int best = 1;
   double best_cost = 1e30;
@@ -91,7 +94,7 @@ int choose_split(int ntiles, int nst_total, int n_ctas, bool force_one) {
     if (nst_total % S) continue;
     const long long tasks = (long long)ntiles * S;
     const long long per = (tasks + n_ctas - 1) / n_ctas;
-    const double cost = per * (nst_total / (double)S + 0.75);
+    const double cost = per * (nst_total / (double)S + 0.75) + (double)S * out_rows * 4.0 / kStageBytes;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = S;
@@ -201,6 +204,7 @@ struct dec_ctx {
   std::vector<void*> allocs;
   size_t bytes_alloc = 0;
   unsigned* d_counters = nullptr;
+  size_t n_counters = 0;
   StepState* d_state = nullptr;
   unsigned* d_started = nullptr;
   Status* d_status = nullptr;
@@ -305,12 +309,18 @@ struct Planner {
   }
 
   // Create a GEMV op over segments sharing K; returns op index.
-  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool force_s1, const char* name) {
+  // whole_reader: every CTA running the consumer reads the whole output (a GEMV prologue);
+  // false when each consumer task reads only its own slice (attention reading q/k/v).
+  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool force_s1, const char* name,
+           bool whole_reader = true) {
     OpDesc o = base_op(OP_GEMV, layer);
     const Geo g = gemv_geometry(K, c->wb);
     int ntiles = 0;
     for (auto& s : segs) ntiles += (s.mat->N + g.R - 1) / g.R;
-    const int S = choose_split(ntiles, g.nst_total, c->n_ctas, force_s1);
+    long long out_rows = 0;
+    if (whole_reader)
+      for (auto& sp : segs) out_rows += sp.mat->N;
+    const int S = choose_split(ntiles, g.nst_total, c->n_ctas, out_rows, force_s1);
     o.wtype = c->wtype;
     o.K = K;
     o.Kpad = g.Kpad;
@@ -463,7 +473,7 @@ static int build_plan(dec_ctx* c) {
       Mat* wq = P.new_mat(DEC_W_Q, l, hq * hd, d, 1, 0);
       Mat* wk = P.new_mat(DEC_W_K, l, hkv * hd, d, 1, 0);
       Mat* wv = P.new_mat(DEC_W_V, l, hkv * hd, d, 1, 0);
-      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv");
+      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv", false);
       if (qkv < 0) return P.rc;
       {
         OpDesc& o = c->ops[qkv];
@@ -495,6 +505,7 @@ static int build_plan(dec_ctx* c) {
       a.m_out = attn_buf[0];
       a.l_out = attn_buf[1];
       a.o_out = attn_buf[2];
+      if (dalloc(c, &a.o_fin, (size_t)hq * hd * 4)) return DEC_ERR_OOM;
       a.kcache = c->kc[l];
       a.vcache = c->vc[l];
       a.rope_cos = c->rope_cos;
@@ -504,14 +515,9 @@ static int build_plan(dec_ctx* c) {
       o_op = P.gemv({{wo, -1, 0}}, hq * hd, l, false, "o_proj");
       if (o_op < 0) return P.rc;
       OpDesc& oo = c->ops[o_op];
-      oo.pro = PRO_ATTN_COMBINE;
+      oo.pro = PRO_SUM;  // the attention op's last chunk task per kv head combined the chunks
       oo.n = hq * hd;
-      oo.am = attn_buf[0];
-      oo.al = attn_buf[1];
-      oo.ao = attn_buf[2];
-      oo.nch = a.nch;
-      oo.nheads = hq;
-      oo.hdim = hd;
+      oo.src = PSet{c->ops[attn].o_fin, 1, hq * hd, 0};
       oo.dep[0] = attn;
     } else {
       const int H = f.n_heads, nope = f.qk_nope, rd = f.qk_rope, vh = f.v_head, kvl = f.kv_lora;
@@ -951,10 +957,24 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
       if (o.router) o.route_dump = c->d_route_dump + f.top_k * i++;
   }
   // per op: the dependency counter, then (routers) the finished-task counter
-  if ((rc = dalloc(c, &c->d_counters, c->ops.size() * 8))) return rc;
-  CK(cudaMemsetAsync(c->d_counters, 0, c->ops.size() * 8, c->stream));
-  for (size_t i = 0; i < c->ops.size(); ++i)
-    if (c->ops[i].router) c->ops[i].fin = c->d_counters + c->ops.size() + i;
+  // per op: the dependency counter and the router's finished-task counter; per dense
+  // attention op: one finished-task counter per kv head. All reset together.
+  c->n_counters = 2 * c->ops.size();
+  for (auto& o : c->ops)
+    if (o.kind == OP_ATTN) c->n_counters += o.hkv;
+  if ((rc = dalloc(c, &c->d_counters, c->n_counters * 4))) return rc;
+  CK(cudaMemsetAsync(c->d_counters, 0, c->n_counters * 4, c->stream));
+  {
+    unsigned* next = c->d_counters + 2 * c->ops.size();
+    for (size_t i = 0; i < c->ops.size(); ++i) {
+      OpDesc& o = c->ops[i];
+      if (o.router) o.fin = c->d_counters + c->ops.size() + i;
+      if (o.kind == OP_ATTN) {
+        o.fin = next;
+        next += o.hkv;
+      }
+    }
+  }
   if ((rc = upload_ops(c))) return rc;
   if ((rc = assign_tasks(c))) return rc;
   if ((rc = dalloc(c, &c->d_state, sizeof(StepState)))) return rc;
@@ -1010,7 +1030,7 @@ extern "C" int dec_reset(dec_ctx* c) {
   CK(cudaSetDevice(c->cfg.device));
   cudaStreamSynchronize(c->stream);
   (void)cudaGetLastError();
-  CK(cudaMemsetAsync(c->d_counters, 0, c->ops.size() * 8, c->stream));
+  CK(cudaMemsetAsync(c->d_counters, 0, c->n_counters * 4, c->stream));
   CK(cudaMemsetAsync(c->d_started, 0, 4, c->stream));
   CK(cudaMemsetAsync(c->d_status, 0, sizeof(Status), c->stream));
   StepState st{1, 0, 0, 0};

@@ -148,6 +148,8 @@ struct alignas(16) OpDesc {
   float* m_out;
   float* l_out;
   float* o_out;
+  float* o_fin;  // dense: combined attention output [hq][hd] (the last chunk task of a kv head writes it;
+                 // `fin` then holds one finished-task counter per kv head)
   int np;  // positions per ring stage
   // ---- final op
   const unsigned long long* fin_best;

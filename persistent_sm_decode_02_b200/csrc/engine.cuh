@@ -43,7 +43,7 @@ struct Misc {
   uint64_t fin_bar;          // every MMA completed before TMEM is freed
   uint32_t tmem;             // TMEM base address (MLA engine instances)
   int prod_dep_op;           // op whose producer dependency the producer already waited for
-  int last_task;             // the current router task is the op's last one to finish
+  int last_task;             // the current task is the last of its op (router) or kv head (attention) to finish
   StepState st;
   volatile int abort;
   int x_op, x_group;     // identity of the input vector currently in the work area
@@ -478,23 +478,21 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
                         wt + h * od.nch);
       named_bar_sync(1, kConsumers);
       const int hd = od.hdim;
+      // MLA blocks past position pos hold no partials
+      const int nc = mla ? min(od.nch, m->st.pos / kMlaBlock + 1) : od.nch;
       for (int e = 4 * tid; e < n; e += 4 * kConsumers) {
         const int h = e / hd, d = e % hd;
         const float* w = wt + h * od.nch;
         const float* src = od.ao + ((size_t)(h0 + h) * od.nch) * hd + d;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        int c = 0;
-        // MLA blocks past position pos hold no partials
-        const int nc = mla ? min(od.nch, m->st.pos / kMlaBlock + 1) : od.nch;
-        for (; c + 4 <= nc; c += 4) {
-          const float4 a0 = ldcg4(src + (size_t)c * hd), a1 = ldcg4(src + (size_t)(c + 1) * hd);
-          const float4 a2 = ldcg4(src + (size_t)(c + 2) * hd), a3 = ldcg4(src + (size_t)(c + 3) * hd);
-          fma4(acc, w[c], a0);
-          fma4(acc, w[c + 1], a1);
-          fma4(acc, w[c + 2], a2);
-          fma4(acc, w[c + 3], a3);
+        for (int c0 = 0; c0 < nc; c0 += 8) {  // 8 chunk loads in flight per thread
+          float4 a[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a[u] = c0 + u < nc ? ldcg4(src + (size_t)(c0 + u) * hd) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (c0 + u < nc) fma4(acc, w[c0 + u], a[u]);
         }
-        for (; c < nc; ++c) fma4(acc, w[c], ldcg4(src + (size_t)c * hd));
         store_x4(x, bf, e, acc);
       }
       break;
@@ -950,13 +948,52 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
       mr[h] = mn;
     }
   };
+  // two positions per step: independent loads, dots and butterflies overlap, and one
+  // correction factor serves both
+  auto position2 = [&](const uint8_t* k0, const uint8_t* v0, const uint8_t* k1, const uint8_t* v1, bool two) {
+    float ka[DPL], va[DPL], kb[DPL], vb[DPL], xa[HW], xb[HW];
+    load_dims<DPL>(k0, cbf, lane, ka);
+    load_dims<DPL>(v0, cbf, lane, va);
+    load_dims<DPL>(k1, cbf, lane, kb);
+    load_dims<DPL>(v1, cbf, lane, vb);
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+      float x = 0.f, y = 0.f;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) {
+        x = fmaf(q[h][d], ka[d], x);
+        y = fmaf(q[h][d], kb[d], y);
+      }
+      xa[h] = x;
+      xb[h] = y;
+    }
+    const float ma = group_reduce<HW>(xa, lane);
+    const float mb = group_reduce<HW>(xb, lane);
+#pragma unroll
+    for (int h = 0; h < HW; ++h) {
+      const float sa = __shfl_sync(0xffffffffu, ma, group_holder<HW>(h)) * sl2;
+      const float sbv = __shfl_sync(0xffffffffu, mb, group_holder<HW>(h)) * sl2;
+      const float sb = two ? sbv : -INFINITY;
+      const float mn = fmaxf(mr[h], fmaxf(sa, sb));
+      const float corr = ex2_approx(mr[h] - mn), pa = ex2_approx(sa - mn), pb = ex2_approx(sb - mn);
+      lr[h] = lr[h] * corr + pa + pb;
+#pragma unroll
+      for (int d = 0; d < DPL; ++d) o[h][d] = fmaf(pb, vb[d], fmaf(pa, va[d], o[h][d] * corr));
+      mr[h] = mn;
+    }
+  };
   const int nst = (b.tc - b.t0 + np - 1) / np;
   for (int st = 0; st < nst; ++st) {
     wait_full(P, S, g, op, t);
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
     const int a = b.t0 + st * np;
     const int n = (b.tc - a) < np ? (b.tc - a) : np;
-    for (int tt = wi; tt < n; tt += WPS) position(stage + (size_t)tt * rowb, stage + (size_t)(np + tt) * rowb);
+    for (int tt = wi; tt < n; tt += 2 * WPS) {
+      const bool two = tt + WPS < n;
+      const int t2 = two ? tt + WPS : tt;  // a lone position reads its own row twice, weight 0
+      position2(stage + (size_t)tt * rowb, stage + (size_t)(np + tt) * rowb, stage + (size_t)t2 * rowb,
+                stage + (size_t)(np + t2) * rowb, two);
+    }
     release_stage(S, g);
     ++g;
   }
@@ -994,7 +1031,35 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
       od.l_out[pi] = l;
     }
   }
-  named_bar_sync(1, kConsumers);  // the merge area is free again
+  // The task that finishes the kv head's chunks last combines them once (split-KV
+  // log-sum-exp), so that the output projection reads one vector instead of every chunk.
+  __threadfence();
+  named_bar_sync(1, kConsumers);  // also: the merge area is free again
+  if (tid == 0) m->last_task = atomicAdd(od.fin + kvh, 1u) + 1 == (unsigned)m->st.epoch * (unsigned)nch;
+  named_bar_sync(1, kConsumers);
+  if (m->last_task) {
+    __threadfence();
+    float* wt = reinterpret_cast<float*>(S.work + kCombineOff);  // [gs][nch]
+    if (warp < gs) {
+      const int qh = kvh * gs + warp;
+      combine_weights(od.m_out + (size_t)qh * nch, od.l_out + (size_t)qh * nch, nch, wt + warp * nch);
+    }
+    named_bar_sync(1, kConsumers);
+    for (int e = tid; e < gs * hd; e += kConsumers) {
+      const int h = e / hd, d = e % hd, qh = kvh * gs + h;
+      const float* src = od.o_out + (size_t)qh * nch * hd + d;
+      float acc = 0.f;
+      for (int c0 = 0; c0 < nch; c0 += 8) {
+        float a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a[u] = c0 + u < nch ? ldcg(src + (size_t)(c0 + u) * hd) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (c0 + u < nch) acc = fmaf(wt[h * nch + c0 + u], a[u], acc);
+      }
+      od.o_fin[(size_t)qh * hd + d] = acc;
+    }
+  }
 }
 
 template <int DPL>
