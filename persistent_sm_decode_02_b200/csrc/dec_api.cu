@@ -566,6 +566,11 @@ static int build_plan(dec_ctx* c) {
         o.rdim = rd;
         o.rope_cos = c->rope_cos;
         o.rope_sin = c->rope_sin;
+        // its first task also appends the step's latent row (normalised c, RoPE'd k_pe) to the cache
+        const OpDesc& p1 = c->ops[s1];
+        o.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
+        o.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
+        o.kcache = c->kc[l];
       }
       OpDesc a = P.base_op(OP_MLA, l);
       {

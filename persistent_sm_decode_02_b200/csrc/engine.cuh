@@ -485,14 +485,16 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         const float* w = wt + h * od.nch;
         const float* src = od.ao + ((size_t)(h0 + h) * od.nch) * hd + d;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c0 = 0; c0 < nc; c0 += 8) {  // 8 chunk loads in flight per thread
-          float4 a[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) a[u] = c0 + u < nc ? ldcg4(src + (size_t)(c0 + u) * hd) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (c0 + u < nc) fma4(acc, w[c0 + u], a[u]);
+        int c = 0;
+        for (; c + 4 <= nc; c += 4) {
+          const float4 a0 = ldcg4(src + (size_t)c * hd), a1 = ldcg4(src + (size_t)(c + 1) * hd);
+          const float4 a2 = ldcg4(src + (size_t)(c + 2) * hd), a3 = ldcg4(src + (size_t)(c + 3) * hd);
+          fma4(acc, w[c], a0);
+          fma4(acc, w[c + 1], a1);
+          fma4(acc, w[c + 2], a2);
+          fma4(acc, w[c + 3], a3);
         }
+        for (; c < nc; ++c) fma4(acc, w[c], ldcg4(src + (size_t)c * hd));
         store_x4(x, bf, e, acc);
       }
       break;
@@ -708,6 +710,42 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
   }
 }
 
+// MLA: the step's new latent cache row, c = bf16(RMSNorm(kv_a latent) * g) and
+// k_pe = bf16(RoPE(kv_a rope part)), stored at position pos of the blocked cache
+// (all consumer threads; absorb_q's first task, before attention reads the block).
+__device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
+  Misc* m = S.m;
+  const int tid = threadIdx.x, pos = m->st.pos;
+  const int kvl = od.rows_per_group, rd = od.rdim, rowe = kvl + rd;
+  __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(S.work + kCombineOff);  // [rowe]
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (4 * tid < kvl) v = pset4(od.ckv, 4 * tid);  // 16-byte loads of the split partials
+  const float tot = consumer_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, m);
+  const float inv = 1.0f / sqrtf(tot / (float)kvl + od.eps);
+  if (4 * tid < kvl) {
+    const float4 g4 = __ldg(reinterpret_cast<const float4*>(od.kvnorm_g + 4 * tid));
+    reinterpret_cast<__nv_bfloat162*>(row)[2 * tid] = __floats2bfloat162_rn(v.x * inv * g4.x, v.y * inv * g4.y);
+    reinterpret_cast<__nv_bfloat162*>(row)[2 * tid + 1] = __floats2bfloat162_rn(v.z * inv * g4.z, v.w * inv * g4.w);
+  }
+  const int rq = tid - kvl / 4;  // RoPE: 4 pairs (j, j + rd/2) per thread
+  if (rq >= 0 && 4 * rq < rd / 2) {
+    const int j = 4 * rq;
+    const float4 a = pset4(od.ckv, kvl + j), b = pset4(od.ckv, kvl + j + rd / 2);
+    const float4 cs = __ldg(reinterpret_cast<const float4*>(od.rope_cos + (size_t)pos * (rd / 2) + j));
+    const float4 sn = __ldg(reinterpret_cast<const float4*>(od.rope_sin + (size_t)pos * (rd / 2) + j));
+    __nv_bfloat162* lo = reinterpret_cast<__nv_bfloat162*>(row + kvl + j);
+    __nv_bfloat162* hi = reinterpret_cast<__nv_bfloat162*>(row + kvl + j + rd / 2);
+    lo[0] = __floats2bfloat162_rn(a.x * cs.x - b.x * sn.x, a.y * cs.y - b.y * sn.y);
+    lo[1] = __floats2bfloat162_rn(a.z * cs.z - b.z * sn.z, a.w * cs.w - b.w * sn.w);
+    hi[0] = __floats2bfloat162_rn(a.x * sn.x + b.x * cs.x, a.y * sn.y + b.y * cs.y);
+    hi[1] = __floats2bfloat162_rn(a.z * sn.z + b.z * cs.z, a.w * sn.w + b.w * cs.w);
+  }
+  named_bar_sync(1, kConsumers);
+  uint8_t* blk = reinterpret_cast<uint8_t*>(od.kcache) + (size_t)(pos / kMlaBlock) * rowe * kMlaBlock * 2;
+  for (int k = tid; k < rowe / 8; k += kConsumers)
+    *reinterpret_cast<uint4*>(blk + mla_cache_off(pos % kMlaBlock, 8 * k)) = reinterpret_cast<const uint4*>(row)[k];
+}
+
 template <int WT>
 __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
                                              uint32_t& g) {
@@ -747,6 +785,7 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
     }
   }
   if (od.qc) {
+    if (t == 0) mla_new_row(od, S);
     // absorb_q also feeds the tensor-core MLA attention: gemv_task stored q_lat
     // rows in bf16; the first tile of head h adds its RoPE'd q_pe (bf16).
     if (geo.s == 0 && (geo.rt * od.R) % od.rows_per_group == 0) {
@@ -1095,9 +1134,8 @@ __device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od,
 //   O = P . C_lat : two ring stages of 256 latent dims (32 KB each); C is
 //                 read MN-major from the same bytes the S step read K-major.
 // The task publishes (m, l, O) for the split-KV log-sum-exp combine in the uv
-// projection's prologue.  The block holding position pos also normalises and
-// RoPEs the step's new latent row, stores it in the cache and patches it into
-// each stage before the MMAs read the stage.
+// projection's prologue.  The step's new latent row is already in the cache:
+// absorb_q's first task writes it (mla_new_row).
 // TMEM: 512 fp32 columns x 128 lanes; S uses columns 0..63 and is read out
 // before O (columns 0..511) overwrites it.
 __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g,
@@ -1114,43 +1152,9 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     return;
   }
   const int n = T - t0 < kMlaBlock ? T - t0 : kMlaBlock;
-  const bool has_new = pos < t0 + kMlaBlock;
-  const int pin = pos - t0;
   const int kvl = od.kvl, rd = od.rdim, rowe = kvl + rd;
   uint8_t* Phi = S.work;                                                   // [64 pos] x [128 heads] bf16, A layout
   uint8_t* Plo = S.work + 16384;
-  __nv_bfloat16* newrow = reinterpret_cast<__nv_bfloat16*>(S.work + 32768);  // [rowe]
-  const long long blk_bytes = (long long)rowe * kMlaBlock * 2;
-  uint8_t* blk = reinterpret_cast<uint8_t*>(od.kcache) + (size_t)c * blk_bytes;
-  if (has_new) {
-    // c = bf16(RMSNorm(kv_a latent) * g); k_pe = bf16(RoPE(kv_a rope part)); 16-byte loads of the split partials
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (4 * tid < kvl) v = pset4(od.ckv, 4 * tid);
-    const float tot = consumer_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, m);
-    const float inv = 1.0f / sqrtf(tot / (float)kvl + od.eps);
-    if (4 * tid < kvl) {
-      const float4 g4 = __ldg(reinterpret_cast<const float4*>(od.kvnorm_g + 4 * tid));
-      reinterpret_cast<__nv_bfloat162*>(newrow)[2 * tid] = __floats2bfloat162_rn(v.x * inv * g4.x, v.y * inv * g4.y);
-      reinterpret_cast<__nv_bfloat162*>(newrow)[2 * tid + 1] = __floats2bfloat162_rn(v.z * inv * g4.z, v.w * inv * g4.w);
-    }
-    const int rq = tid - kvl / 4;  // RoPE: 4 pairs (j, j + rd/2) per thread
-    if (rq >= 0 && 4 * rq < rd / 2) {
-      const int j = 4 * rq;
-      const float4 a = pset4(od.ckv, kvl + j), b = pset4(od.ckv, kvl + j + rd / 2);
-      const float4 cs = __ldg(reinterpret_cast<const float4*>(od.rope_cos + (size_t)pos * (rd / 2) + j));
-      const float4 sn = __ldg(reinterpret_cast<const float4*>(od.rope_sin + (size_t)pos * (rd / 2) + j));
-      __nv_bfloat162* lo = reinterpret_cast<__nv_bfloat162*>(newrow + kvl + j);
-      __nv_bfloat162* hi = reinterpret_cast<__nv_bfloat162*>(newrow + kvl + j + rd / 2);
-      lo[0] = __floats2bfloat162_rn(a.x * cs.x - b.x * sn.x, a.y * cs.y - b.y * sn.y);
-      lo[1] = __floats2bfloat162_rn(a.z * cs.z - b.z * sn.z, a.w * cs.w - b.w * sn.w);
-      hi[0] = __floats2bfloat162_rn(a.x * sn.x + b.x * cs.x, a.y * sn.y + b.y * cs.y);
-      hi[1] = __floats2bfloat162_rn(a.z * sn.z + b.z * cs.z, a.w * sn.w + b.w * cs.w);
-    }
-    named_bar_sync(1, kConsumers);
-    // append to the cache (read by later steps only)
-    for (int k = tid; k < rowe / 8; k += kConsumers)
-      *reinterpret_cast<uint4*>(blk + mla_cache_off(pin, 8 * k)) = reinterpret_cast<const uint4*>(newrow)[k];
-  }
   const uint32_t tm = m->tmem;
   constexpr uint32_t kIdS = umma_idesc_bf16(128, kMlaBlock, false);
   constexpr uint32_t kIdO = umma_idesc_bf16(128, 256, true);
@@ -1159,13 +1163,6 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   for (int j = 0; j < nS; ++j) {
     wait_full(P, S, g, op, t);
     uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    if (has_new) {  // the new row's 64 dims of this chunk
-      if (tid < 8)
-        *reinterpret_cast<uint4*>(stage + 16384 + mla_cache_off(pin, 8 * tid)) =
-            reinterpret_cast<const uint4*>(newrow)[8 * j + tid];
-      fence_async_smem();
-      named_bar_sync(1, kConsumers);
-    }
     if (warp == 0) {
       if (lane == 0) {
         tc_fence_after();
@@ -1238,12 +1235,6 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   for (int o = 0; o < kvl / 256; ++o) {
     wait_full(P, S, g, op, t);
     uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    if (has_new) {
-      if (tid < 32)
-        *reinterpret_cast<uint4*>(stage + mla_cache_off(pin, 8 * tid)) = reinterpret_cast<const uint4*>(newrow)[32 * o + tid];
-      fence_async_smem();
-      named_bar_sync(1, kConsumers);
-    }
     if (warp == 0) {
       if (lane == 0) {
         tc_fence_after();
@@ -1267,7 +1258,7 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   __syncwarp();
   tc_fence_after();
   const int col0 = 256 * half;
-  float* tile = reinterpret_cast<float*>(S.work) + warp * (32 * 36);  // [32 heads][36] (P and newrow are dead)
+  float* tile = reinterpret_cast<float*>(S.work) + warp * (32 * 36);  // [32 heads][36] (P is dead)
 #pragma unroll 1
   for (int cc = 0; cc < 8; ++cc) {
     uint32_t r[32];
@@ -1392,7 +1383,7 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
       uint8_t* dst = S.ring + (g % kStages) * kStageBytes;
       uint64_t* fb = &m->full[g % kStages];
       mbar_arrive_expect_tx(fb, bytes + bytes2);
-      if (bytes) bulk_g2s(dst, src, bytes, fb, pol);
+      if (bytes && src) bulk_g2s(dst, src, bytes, fb, pol);  // src null: the caller copies it later
       if (bytes2) bulk_g2s(dst + off2, src2, bytes2, fb, pol);
     }
     __syncwarp();
@@ -1452,9 +1443,20 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
     } else if (od.kind == OP_MLA) {
       // block t: nine (Q chunk, C chunk) stages for S, then two C stages for O
       if (t * kMlaBlock <= pos) {
-        if (m->prod_dep_op != op) {  // the absorbed query is written by the absorb_q op
-          int r = 1;
-          if (lane == 0) {
+        const int rowe = od.kvl + od.rdim, nS = rowe / 64;
+        const uint8_t* blk = (const uint8_t*)od.kcache + (size_t)t * rowe * kMlaBlock * 2;
+        const uint8_t* q = (const uint8_t*)od.qc;
+        int early = 0;
+        const uint32_t g0 = g;
+        if (m->prod_dep_op != op) {
+          // The cache chunks do not depend on this step's ops (except in the block that
+          // absorb_q appends to): start them in the first free stages now; the query
+          // chunks (written by absorb_q) join the same stages once absorb_q is done.
+          if (pos >= (t + 1) * kMlaBlock)
+            for (; early < nS && early < kStages && ok; ++early)
+              ok = issue(nullptr, 16384, blk + early * 8192, 8192, 16384, pol_kv);  // expects both parts
+          int r = ok ? 1 : 0;
+          if (lane == 0 && ok) {
             if (P.persistent) r = wait_counter(P, od.pdep, epoch, &m->abort, op, t) ? 1 : 0;
             fence_async_global();
           }
@@ -1462,13 +1464,16 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
             ok = false;
             break;
           }
-          if (lane == 0) m->prod_dep_op = op;
+          if (lane == 0) {
+            m->prod_dep_op = op;
+            for (int j = 0; j < early; ++j) {
+              const uint32_t gj = g0 + j;
+              bulk_g2s(S.ring + (gj % kStages) * kStageBytes, q + j * 16384, 16384, &m->full[gj % kStages], pol_kv);
+            }
+          }
           __syncwarp();
         }
-        const int rowe = od.kvl + od.rdim;
-        const uint8_t* blk = (const uint8_t*)od.kcache + (size_t)t * rowe * kMlaBlock * 2;
-        const uint8_t* q = (const uint8_t*)od.qc;
-        for (int j = 0; j < rowe / 64 && ok; ++j) ok = issue(q + j * 16384, 16384, blk + j * 8192, 8192, 16384, pol_kv);
+        for (int j = early; j < nS && ok; ++j) ok = issue(q + j * 16384, 16384, blk + j * 8192, 8192, 16384, pol_kv);
         for (int o = 0; o < od.kvl / 256 && ok; ++o) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
       }
     }
