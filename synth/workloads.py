@@ -68,6 +68,12 @@ WORKLOADS = {
     "small_dense_fp8": dict(_BASE_DENSE, n_layers=2, d_model=384, n_heads=4, n_kv_heads=2, head_dim=128,
                             ffn_hidden=1040, vocab=1000, weight_dtype="fp8", ctx=150, n_decode=6, seed=2003,
                             cache_from="oracle"),
+    "small_dense_g8_bf16": dict(_BASE_DENSE, n_layers=2, d_model=512, n_heads=16, n_kv_heads=2, head_dim=128,
+                                ffn_hidden=1024, vocab=1000, weight_dtype="bf16", ctx=90, n_decode=6, seed=2005,
+                                cache_from="oracle"),
+    "small_dense_g8_fp8_hd64": dict(_BASE_DENSE, n_layers=2, d_model=512, n_heads=8, n_kv_heads=1, head_dim=64,
+                                    ffn_hidden=1024, vocab=1000, weight_dtype="fp8", ctx=70, n_decode=6, seed=2006,
+                                    cache_from="oracle"),
     "small_mla_moe_fp8": dict(_BASE_MLA, n_layers=3, d_model=512, n_heads=16, q_lora=384, n_dense_layers=1,
                               ffn_hidden=1024, n_experts=16, top_k=4, expert_hidden=256, vocab=1000,
                               weight_dtype="fp8", ctx=100, n_decode=6, seed=2004, cache_from="oracle"),

@@ -1,7 +1,7 @@
 """GPU decode step vs the CPU oracle, teacher-forced, through the C ABI.
 
 Small workloads (several tiles per op, ragged rows and columns, GQA groups of
-1, 3 and 4, MLA + routed MoE) run every decode step of the workload in all
+1, 2, 3 and 8 with head_dim 64 and 128, MLA + routed MoE) run every decode step of the workload in all
 three execution modes; the persistent kernel, the per-op launches and the CUDA
 graph must agree bit for bit, and each must match the oracle within the
 tolerances of the model definition:
@@ -19,7 +19,8 @@ from synth import workloads
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["tiny_dense_f32", "small_dense_bf16", "small_dense_fp8", "small_mla_moe_fp8"]
+SMALL = ["tiny_dense_f32", "small_dense_bf16", "small_dense_fp8", "small_dense_g8_bf16", "small_dense_g8_fp8_hd64",
+         "small_mla_moe_fp8"]
 MARGIN = 1e-4
 
 
