@@ -158,6 +158,24 @@ def oracle_steps(w, n_steps: int, budget_s: float):
                 cores=om.get_threads())
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, dist=None, device: str = "cuda") -> float:
+    """The largest value of x over all ranks (every rank gets it); x itself without a process group."""
+    if dist is None:
+        return x
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps_per_rank: int, seconds_max: float) -> float:
+    """Whole-job tokens/s: every rank decodes steps_per_rank tokens of its own replica; the job
+    takes as long as its slowest rank."""
+    return world * steps_per_rank / seconds_max
+
+
 # --------------------------------------------------------------------------- GPU arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -198,11 +216,8 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         dec.sync()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1)
+        ms = max_over_ranks(e0.elapsed_time(e1), dist)
         if dist is not None:
-            t = torch.tensor([ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
         return ms
 
@@ -227,11 +242,7 @@ def run_ours(args, rank, world, local_rank):
     t0 = time.perf_counter()
     for _ in range(args.e2e_steps):
         tok = dec.step(tok)
-    e2e_s = time.perf_counter() - t0
-    if dist is not None:
-        t = torch.tensor([e2e_s], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(time.perf_counter() - t0, dist)
 
     T_mean = w["ctx"] + args.warmup + args.steps / 2.0
     bytes_step = workloads.active_bytes_per_token(w, T_mean)["total"]
@@ -242,7 +253,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         result = {
             "metric": METRIC,
-            "value": world * args.steps / (ms_main / 1e3),
+            "value": job_throughput(world, args.steps, ms_main / 1e3),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -265,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
                          "bytes_per_step": bytes_step, "frac_of_8tbs": achieved / 8000.0,
                          "kernel": "engine_kernel (one persistent launch per step)"},
             "clocks": clk,
-            "e2e": {"value": world * args.e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 4,
+            "e2e": {"value": job_throughput(world, args.e2e_steps, e2e_s), "unit": "tokens/s", "h2d_bytes_per_step": 4,
                     "d2h_bytes_per_step": 32, "note": "dec_step: token id in, status + step state (greedy token) out"},
             "gpu_launches": args.steps,
             "ablation": ablation or None,
