@@ -405,6 +405,18 @@ static size_t mla_cache_bytes(const dec_config& f) {
   return (size_t)((f.max_seq + kMlaBlock - 1) / kMlaBlock) * kMlaBlock * (f.kv_lora + f.qk_rope) * 2;
 }
 
+// Grouped GEMVs whose row tiles are tiny (absorb_q: 16 KB, uv: 32 KB per tile) run a whole
+// input group (one head) per task: the prologue and the task overhead are paid once per head.
+static void group_tasks(OpDesc& o) {
+  if (o.kind != OP_GEMV || o.S != 1 || o.rows_per_group <= 0 || o.rows_per_group % o.R) return;
+  const int tpt = o.rows_per_group / o.R;
+  if (tpt <= 1 || o.ntasks % tpt) return;
+  for (int i = 0; i < o.nsegs; ++i)
+    if (o.seg[i].ntiles % tpt || o.seg[i].task0 % tpt) return;
+  o.tpt = tpt;
+  o.ntasks /= tpt;
+}
+
 static float* gainp(dec_ctx* c, int kind, int layer) { return c->vecs[{kind, layer}].p; }
 
 static int build_plan(dec_ctx* c) {
@@ -571,6 +583,8 @@ static int build_plan(dec_ctx* c) {
         o.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
         o.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
         o.kcache = c->kc[l];
+        group_tasks(o);
+        o.ntasks += 1;  // the last task appends the step's latent row (on a CTA with no GEMV task here)
       }
       OpDesc a = P.base_op(OP_MLA, l);
       {
@@ -618,6 +632,7 @@ static int build_plan(dec_ctx* c) {
         o.hdim = kvl;
         o.rows_per_group = vh;
         o.dep[0] = attn;
+        group_tasks(o);
       }
       Mat* wo = P.new_mat(DEC_W_O, l, d, H * vh, 1, 0);
       o_op = P.gemv({{wo, -1, 0}}, H * vh, l, false, "o_proj");

@@ -98,6 +98,7 @@ struct alignas(16) OpDesc {
   int nsegs;
   Seg seg[kMaxSegs];
   int rows_per_group;  // grouped GEMV: input group = row / rows_per_group (0: one input for all rows)
+  int tpt;             // GEMV units (row tile x split) per task (0 or 1: one); a task's units share a group
   void* qc;            // MLA: absorbed bf16 query in the tensor-core layout (written by absorb_q, read by attention)
   float* out;          // fp32 partial outputs [S][out_stride]
   int out_stride;

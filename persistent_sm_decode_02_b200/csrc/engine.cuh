@@ -747,27 +747,41 @@ __device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
 }
 
 template <int WT>
+__device__ __forceinline__ void gemv_unit(const KParams& P, const OpDesc& od, int op, int u, const Smem& S,
+                                          uint32_t& g, const TaskGeo& geo) {
+  switch (od.kcb) {
+    case 4096: gemv_task<WT, 4096>(P, od, op, u, S, g, geo); break;
+    case 2048: gemv_task<WT, 2048>(P, od, op, u, S, g, geo); break;
+    case 1024: gemv_task<WT, 1024>(P, od, op, u, S, g, geo); break;
+    case 512: gemv_task<WT, 512>(P, od, op, u, S, g, geo); break;
+    case 256: gemv_task<WT, 256>(P, od, op, u, S, g, geo); break;
+    case 128: gemv_task<WT, 128>(P, od, op, u, S, g, geo); break;
+    case 64: gemv_task<WT, 64>(P, od, op, u, S, g, geo); break;
+    default: gemv_task<WT, 32>(P, od, op, u, S, g, geo); break;
+  }
+}
+
+template <int WT>
 __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
                                              uint32_t& g) {
-  const TaskGeo geo = gemv_geo(od, t);
   Misc* m = S.m;
+  if (od.qc && t == od.ntasks - 1) {  // absorb_q's extra task: the step's latent cache row
+    mla_new_row(od, S);
+    fence_async_global();  // read by bulk copies of other CTAs after the op's counter
+    return;
+  }
+  const int tpt = od.tpt > 1 ? od.tpt : 1;
+  for (int i = 0; i < tpt; ++i) {  // a task's units (row tiles) share the input group
+  const int u = t * tpt + i;
+  const TaskGeo geo = gemv_geo(od, u);
   if (m->x_op != op || m->x_group != geo.group) {
-    prologue(od, geo.group, t, S);
+    prologue(od, geo.group, u, S);
     if (threadIdx.x == 0) {
       m->x_op = op;
       m->x_group = geo.group;
     }
   }
-  switch (od.kcb) {
-    case 4096: gemv_task<WT, 4096>(P, od, op, t, S, g, geo); break;
-    case 2048: gemv_task<WT, 2048>(P, od, op, t, S, g, geo); break;
-    case 1024: gemv_task<WT, 1024>(P, od, op, t, S, g, geo); break;
-    case 512: gemv_task<WT, 512>(P, od, op, t, S, g, geo); break;
-    case 256: gemv_task<WT, 256>(P, od, op, t, S, g, geo); break;
-    case 128: gemv_task<WT, 128>(P, od, op, t, S, g, geo); break;
-    case 64: gemv_task<WT, 64>(P, od, op, t, S, g, geo); break;
-    default: gemv_task<WT, 32>(P, od, op, t, S, g, geo); break;
-  }
+  gemv_unit<WT>(P, od, op, u, S, g, geo);
   if (od.router) {
     // The task that finishes the router op last sums the logits' split-K
     // partials and stores the top-k ids and weights once for all readers.
@@ -785,7 +799,6 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
     }
   }
   if (od.qc) {
-    if (t == 0) mla_new_row(od, S);
     // absorb_q also feeds the tensor-core MLA attention: gemv_task stored q_lat
     // rows in bf16; the first tile of head h adds its RoPE'd q_pe (bf16).
     if (geo.s == 0 && (geo.rt * od.R) % od.rows_per_group == 0) {
@@ -799,8 +812,9 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
         q[mla_q_off(h, kvl + j + rd / 2) / 2] = __float2bfloat16_rn(a * sn + b * cs);
       }
     }
-    fence_async_global();  // read by bulk copies of other CTAs after the op's counter
   }
+  }  // units
+  if (od.qc) fence_async_global();  // Qc is read by bulk copies of other CTAs after the op's counter
 }
 
 // ------------------------------------------------------- attention tasks
@@ -1406,7 +1420,10 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
       }
     }
     if (od.kind == OP_GEMV) {
-      const TaskGeo geo = gemv_geo(od, t);
+      const int tpt = od.tpt > 1 ? od.tpt : 1;
+      const bool row_task = od.qc && t == od.ntasks - 1;  // absorb_q's latent-row task streams nothing
+      for (int i = 0; i < tpt && ok && !row_task; ++i) {
+      const TaskGeo geo = gemv_geo(od, t * tpt + i);
       const Seg& sg = od.seg[geo.si];
       const uint8_t* base = sg.w;
       if (sg.slot >= 0) {
@@ -1430,6 +1447,7 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
       const uint32_t sb = (uint32_t)(od.R * od.kcb);
       const uint8_t* tile = base + (size_t)(geo.rt * od.S + geo.s) * od.nst * sb;
       for (int st = 0; st < od.nst && ok; ++st) ok = issue(tile + (size_t)st * sb, sb, nullptr, 0, 0, pol_w);
+      }  // units
     } else if (od.kind == OP_ATTN) {
       const int kvh = t / od.nch, c = t % od.nch;
       const ChunkB b = chunk_bounds(c, od.nch, pos);
