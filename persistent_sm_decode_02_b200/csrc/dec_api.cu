@@ -85,7 +85,10 @@ Geo gemv_geometry(int K, int wb) {
 
 // Split-K factor S of a GEMV op, in units of ring stages on the busiest CTA: its tasks'
 // stages plus a fixed cost per task, plus the consumer's prologue, which reads all S
-// partial vectors (out_rows fp32 values each) on every CTA.
+// partial vectors (out_rows fp32 values each) on every CTA.  Every CTA reads the same lines
+// at once, and that L2 read ran about 4x slower per byte than a weight stage in the device
+// trace, hence the weight.
+constexpr double kPrologueWeight = 4.0;
 int choose_split(int ntiles, int nst_total, int n_ctas, long long out_rows, bool force_one) {
   if (force_one) return 1;
   int best = 1;
@@ -94,7 +97,7 @@ int choose_split(int ntiles, int nst_total, int n_ctas, long long out_rows, bool
     if (nst_total % S) continue;
     const long long tasks = (long long)ntiles * S;
     const long long per = (tasks + n_ctas - 1) / n_ctas;
-    const double cost = per * (nst_total / (double)S + 0.75) + (double)S * out_rows * 4.0 / kStageBytes;
+    const double cost = per * (nst_total / (double)S + 0.75) + kPrologueWeight * S * out_rows * 4.0 / kStageBytes;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = S;
@@ -543,7 +546,7 @@ static int build_plan(dec_ctx* c) {
         o.h_out = h_in[l];
       }
       Mat* qb = P.new_mat(DEC_W_Q_B, l, H * (nope + rd), f.q_lora, 1, 0);
-      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b");
+      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b", false);  // absorb_q reads one head per task
       if (s2 < 0) return P.rc;
       {
         OpDesc& o = c->ops[s2];
