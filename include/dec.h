@@ -111,11 +111,14 @@ enum {
 /* ------------------------------------------------------------------ types */
 typedef struct dec_ctx dec_ctx; /* opaque; owns all of its device memory */
 
+/* Limits checked by dec_create (DEC_ERR_UNSUPPORTED otherwise): dense head_dim 64 or 128,
+ * n_heads / n_kv_heads <= 8, n_heads <= 128; MLA kv_lora 512, qk_rope 64 or 128, n_heads <= 128
+ * (the attention's tensor-core tile is 128 heads), bf16 or FP8 weights. */
 typedef struct dec_config {
   int32_t arch;                                          /* DEC_ARCH_* */
   int32_t n_layers, d_model, vocab, max_seq;             /* max_seq: context + generated positions */
   int32_t n_heads, n_kv_heads, head_dim, ffn_hidden;     /* dense attention; ffn_hidden also sizes MLA's dense layers */
-  int32_t q_lora, kv_lora, qk_nope, qk_rope, v_head;     /* MLA (kv_lora 512, qk_nope 128, qk_rope 64, v_head 128) */
+  int32_t q_lora, kv_lora, qk_nope, qk_rope, v_head;     /* MLA (the pages' model: 512, 128, 64, 128) */
   int32_t n_dense_layers, n_experts, top_k, n_shared, expert_hidden; /* MoE */
   float rope_theta, norm_eps;
   int32_t weight_dtype;   /* DEC_F32 | DEC_BF16 | DEC_FP8_E4M3_B128 */

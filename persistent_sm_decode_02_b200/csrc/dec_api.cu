@@ -876,14 +876,13 @@ static int check_work_area(dec_ctx* c) {
     const OpDesc& o = c->ops[i];
     const char* nm = c->op_names[i].c_str();
     if (o.kind != OP_GEMV) continue;
-    const int cap = (o.pro == PRO_ATTN_COMBINE || o.pro == PRO_MLA_COMBINE) ? kCombineOff : kWorkBytes;
+    const int cap = o.pro == PRO_MLA_COMBINE ? kCombineOff : kWorkBytes;
     if ((long long)o.Kpad * (o.in_bf16 ? 2 : 4) > cap)
       return fail(c, DEC_ERR_UNSUPPORTED, "input vector of op %zu (%s) exceeds the work area", i, nm);
     if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.add2) || !al(o.routed) || !al(o.src) || !al(o.gate) ||
         !al(o.up) || o.routed_slot_stride % 4 || o.slot_stride % 4 || o.gstride % 4 || o.hdim % 4)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): vector lengths and offsets must be multiples of 4", i, nm);
-    if ((o.pro == PRO_ATTN_COMBINE && (o.nch > 64 || (long long)o.nheads * o.nch > kMaxCombine)) ||
-        (o.pro == PRO_MLA_COMBINE && o.nch > kMaxCombine))
+    if (o.pro == PRO_MLA_COMBINE && o.nch > kMaxCombine)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): too many split-KV chunks", i, nm);
   }
   return DEC_OK;

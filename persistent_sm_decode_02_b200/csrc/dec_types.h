@@ -66,7 +66,6 @@ enum Pro : int {
   PRO_NORM_SUM = 2,     // x = R(rmsnorm(sum of partials) * g)
   PRO_SUM = 3,          // x = R(sum of partials) (optionally per input group)
   PRO_SWIGLU = 4,       // x = R(silu(gate) * up)
-  PRO_ATTN_COMBINE = 5, // x = R(split-KV log-sum-exp combine) for all heads
   PRO_MLA_COMBINE = 6   // x = R(split-KV combine of one head's latent output)
 };
 

@@ -466,11 +466,9 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
       }
       break;
     }
-    case PRO_ATTN_COMBINE:
     case PRO_MLA_COMBINE: {
-      // per-chunk weights of every head this input needs, then weighted sums of the chunk outputs
-      const bool mla = od.pro == PRO_MLA_COMBINE;
-      const int h0 = mla ? group : 0, nh = mla ? 1 : od.nheads;
+      // per-chunk weights of the group's head, then the weighted sum of its chunk outputs
+      const int h0 = group, nh = 1;
       float* wt = reinterpret_cast<float*>(S.work + kCombineOff);  // [nh][nch]
       const int warp = tid >> 5;
       for (int h = warp; h < nh; h += kConsumerWarps)
@@ -479,7 +477,7 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
       named_bar_sync(1, kConsumers);
       const int hd = od.hdim;
       // MLA blocks past position pos hold no partials
-      const int nc = mla ? min(od.nch, m->st.pos / kMlaBlock + 1) : od.nch;
+      const int nc = min(od.nch, m->st.pos / kMlaBlock + 1);
       for (int e = 4 * tid; e < n; e += 4 * kConsumers) {
         const int h = e / hd, d = e % hd;
         const float* w = wt + h * od.nch;
