@@ -99,3 +99,27 @@ def test_invalid_config_is_rejected_before_any_device_call():
     with pytest.raises(pkg.DecError) as e:
         pkg.Decoder(pkg.config_from_workload(w))
     assert e.value.code == pkg.dec.DEC_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("over", [
+    dict(n_heads=256),                # the tensor-core MLA tile holds 128 heads
+    dict(qk_rope=32),                 # 64-dim K chunks of [latent | rope key]
+    dict(kv_lora=256),
+    dict(weight_dtype="f32"),         # MLA runs on bf16 activations
+])
+def test_mla_limits_are_rejected_before_any_device_call(over):
+    import persistent_sm_decode_02_b200 as pkg
+    from synth import workloads
+    w = workloads.get("small_mla_moe_fp8", **over)
+    with pytest.raises(pkg.DecError) as e:
+        pkg.Decoder(pkg.config_from_workload(w))
+    assert e.value.code == pkg.dec.DEC_ERR_UNSUPPORTED
+
+
+def test_gqa_group_above_eight_is_rejected():
+    import persistent_sm_decode_02_b200 as pkg
+    from synth import workloads
+    w = workloads.get("small_dense_g8_bf16", n_heads=32)  # 32 / 2 = 16 query heads per kv head
+    with pytest.raises(pkg.DecError) as e:
+        pkg.Decoder(pkg.config_from_workload(w))
+    assert e.value.code == pkg.dec.DEC_ERR_UNSUPPORTED
