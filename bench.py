@@ -170,6 +170,15 @@ def max_over_ranks(x: float, dist=None, device: str = "cuda") -> float:
     return float(t.item())
 
 
+def tpot_stats(per_step_ms):
+    """Median, p99 and max of the per-step times (ms) in microseconds (this rank's steps)."""
+    xs = sorted(per_step_ms)
+    if not xs:
+        return None
+    pick = lambda q: xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))]  # nearest rank
+    return {"p50": pick(0.5) * 1e3, "p99": pick(0.99) * 1e3, "max": xs[-1] * 1e3, "steps": len(xs)}
+
+
 def job_throughput(world: int, steps_per_rank: int, seconds_max: float) -> float:
     """Whole-job tokens/s: every rank decodes steps_per_rank tokens of its own replica; the job
     takes as long as its slowest rank."""
@@ -199,6 +208,8 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream()
     dec.set_stream(stream.cuda_stream)
 
+    per_step = {}
+
     def timed_chain(mode):
         dec.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
         dec.set_exec_mode(mode)
@@ -209,14 +220,15 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        ev[0].record(stream)
+        for i in range(args.steps):
             dec.step_async(-1)
-        e1.record(stream)
+            ev[i + 1].record(stream)  # per-step boundaries for the TPOT distribution
         dec.sync()
         torch.cuda.synchronize()
-        ms = max_over_ranks(e0.elapsed_time(e1), dist)
+        per_step[mode] = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+        ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist)
         if dist is not None:
             dist.barrier()
         return ms
@@ -260,6 +272,7 @@ def run_ours(args, rank, world, local_rank):
             "warmup": args.warmup,
             "ms_per_step": ms_step,
             "tpot_us": ms_step * 1e3,
+            "tpot_us_dist": tpot_stats(per_step[pkg.dec.DEC_PERSISTENT]),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,

@@ -79,3 +79,13 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert out.returncode == 0, out.stderr
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_tpot_stats_nearest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    st = bench.tpot_stats([3.0, 1.0, 2.0] + [2.0] * 97)  # ms per step
+    assert st["p50"] == 2000.0 and st["max"] == 3000.0 and st["steps"] == 100
+    assert st["p99"] == 2000.0  # nearest rank of 99 % of 100 steps
+    assert bench.tpot_stats([]) is None
