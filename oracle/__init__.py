@@ -20,6 +20,9 @@ torch.float8_e4m3fn, bf16 rounding against torch, RoPE norm preservation and
 relative-position invariance, incremental decode == full causal recompute,
 context length 1 returns V, one expert with top-1 == the dense MLP, router
 weights sum to 1, absorbed MLA == unabsorbed MLA, split-KV log-sum-exp combine
-== one softmax, argmax == numpy first-max.  Parity of whole-model values beyond
+== one softmax, argmax == numpy first-max; and closed forms of special cases that bypass
+the step code (test_oracle_structure.py): zeroed output projections pass the embedding
+through, a one-layer FFN-only step, two-position attention as a sigmoid mix (dense and MLA),
+two-expert router weights as a sigmoid pair.  Parity of whole-model values beyond
 these pins is unpinned: the pages print no worked example.
 """
