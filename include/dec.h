@@ -142,6 +142,8 @@ typedef struct dec_tensor {
 
 /* Validate the configuration, plan the task list of one decode step and
  * allocate all device memory (weights, caches, activations, counters).
+ * On an error *out may still hold a context that carries the message for
+ * dec_last_error; pass it to dec_destroy, which frees what was allocated.
  * Errors: INVALID_ARG (bad config), UNSUPPORTED, OOM, CUDA. */
 int dec_create(const dec_config* cfg, dec_ctx** out);
 
@@ -189,7 +191,10 @@ int dec_reset(dec_ctx* c);
 int dec_destroy(dec_ctx* c);
 
 /* Use `stream` (a cudaStream_t, NULL = the legacy default stream) for all
- * further work of the context. */
+ * further work of the context, after the work already queued on the current
+ * one has finished.  The caller keeps ownership: the stream must stay valid
+ * until the context is destroyed or given another stream, and dec_destroy
+ * synchronises it but destroys only the stream that dec_create made. */
 int dec_set_stream(dec_ctx* c, void* stream);
 
 /* Switch between DEC_PERSISTENT, DEC_PER_OP and DEC_PER_OP_GRAPH for further

@@ -192,7 +192,8 @@ const void* pick_kernel(int wtype, bool mla) {
 struct dec_ctx {
   dec_config cfg{};
   int n_ctas = 0;
-  cudaStream_t stream = nullptr;
+  cudaStream_t stream = nullptr;      // where the context's work is ordered
+  cudaStream_t own_stream = nullptr;  // the stream dec_create made; the only one dec_destroy destroys
   std::string err = "";
   int wtype = WT_F32, wb = 4, act_bf16 = 0, eb = 4;
   // plan
@@ -924,7 +925,8 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
   CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, c->kernel, kThreads, kSmemBytes));
   if (per_sm < 1 || !coop) return fail(c, DEC_ERR_UNSUPPORTED, "device cannot host the persistent kernel");
   c->n_ctas = f.n_ctas > 0 ? std::min(f.n_ctas, sms * per_sm) : sms;
-  CK(cudaStreamCreateWithFlags(&c->stream, cudaStreamNonBlocking));
+  CK(cudaStreamCreateWithFlags(&c->own_stream, cudaStreamNonBlocking));
+  c->stream = c->own_stream;
   const int L = f.n_layers, d = f.d_model;
   const bool mla = f.arch == DEC_ARCH_MLA_MOE;
   // embedding, gains, caches, RoPE tables (referenced by the plan)
@@ -1021,9 +1023,13 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
 
 extern "C" int dec_destroy(dec_ctx* c) {
   if (!c) return DEC_OK;
-  if (c->stream) cudaStreamSynchronize(c->stream);
+  if (c->own_stream) {  // creation got as far as the stream: the device is set up
+    cudaSetDevice(c->cfg.device);
+    cudaStreamSynchronize(c->stream);
+  }
   free_all(c);
-  if (c->stream) cudaStreamDestroy(c->stream);
+  if (c->own_stream) cudaStreamDestroy(c->own_stream);  // a stream given by dec_set_stream stays the caller's
+  (void)cudaGetLastError();
   delete c;
   return DEC_OK;
 }
@@ -1241,37 +1247,44 @@ extern "C" int dec_set_kv_cache(dec_ctx* c, const void* k_or_latent, const void*
   int rc = dec_reset(c);
   if (rc) return rc;
   const bool mla = f.arch == DEC_ARCH_MLA_MOE;
-  uint8_t* rows = nullptr;
-  for (int l = 0; l < f.n_layers && n_tokens > 0; ++l) {
-    if (!mla) {
-      const size_t row = (size_t)n_tokens * f.head_dim * c->eb;  // one kv head
-      const size_t src_layer = (size_t)f.n_kv_heads * row;
-      const size_t dpitch = (size_t)f.max_seq * f.head_dim * c->eb;
-      CK(cudaMemcpy2DAsync(c->kc[l], dpitch, (const uint8_t*)k_or_latent + l * src_layer, row, row, f.n_kv_heads,
-                           cudaMemcpyDefault, c->stream));
-      CK(cudaMemcpy2DAsync(c->vc[l], dpitch, (const uint8_t*)v_or_pe + l * src_layer, row, row, f.n_kv_heads,
-                           cudaMemcpyDefault, c->stream));
-    } else {  // rows [n][kv_lora | qk_rope] in a scratch buffer, then the blocked layout
-      const size_t lat = (size_t)f.kv_lora * 2, pe = (size_t)f.qk_rope * 2, rowb = lat + pe;
-      if (!rows) {
-        cudaError_t e = cudaMalloc(&rows, (size_t)n_tokens * rowb);
-        if (e != cudaSuccess) {
-          (void)cudaGetLastError();
-          return fail(c, DEC_ERR_OOM, "cache scratch of %zu bytes: %s", (size_t)n_tokens * rowb, cudaGetErrorString(e));
+  uint8_t* rows = nullptr;  // MLA only: [n][kv_lora | qk_rope] rows of one layer, freed on every path
+  auto copy_layers = [&]() -> int {
+    for (int l = 0; l < f.n_layers && n_tokens > 0; ++l) {
+      if (!mla) {
+        const size_t row = (size_t)n_tokens * f.head_dim * c->eb;  // one kv head
+        const size_t src_layer = (size_t)f.n_kv_heads * row;
+        const size_t dpitch = (size_t)f.max_seq * f.head_dim * c->eb;
+        CK(cudaMemcpy2DAsync(c->kc[l], dpitch, (const uint8_t*)k_or_latent + l * src_layer, row, row, f.n_kv_heads,
+                             cudaMemcpyDefault, c->stream));
+        CK(cudaMemcpy2DAsync(c->vc[l], dpitch, (const uint8_t*)v_or_pe + l * src_layer, row, row, f.n_kv_heads,
+                             cudaMemcpyDefault, c->stream));
+      } else {  // rows [n][kv_lora | qk_rope] in a scratch buffer, then the blocked layout
+        const size_t lat = (size_t)f.kv_lora * 2, pe = (size_t)f.qk_rope * 2, rowb = lat + pe;
+        if (!rows) {
+          cudaError_t e = cudaMalloc(&rows, (size_t)n_tokens * rowb);
+          if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            return fail(c, DEC_ERR_OOM, "cache scratch of %zu bytes: %s", (size_t)n_tokens * rowb, cudaGetErrorString(e));
+          }
         }
+        CK(cudaMemcpy2DAsync(rows, rowb, (const uint8_t*)k_or_latent + (size_t)l * n_tokens * lat, lat, lat, n_tokens,
+                             cudaMemcpyDefault, c->stream));
+        CK(cudaMemcpy2DAsync(rows + lat, rowb, (const uint8_t*)v_or_pe + (size_t)l * n_tokens * pe, pe, pe, n_tokens,
+                             cudaMemcpyDefault, c->stream));
+        mla_cache_convert<<<1184, 256, 0, c->stream>>>(rows, (uint8_t*)c->kc[l], n_tokens, f.kv_lora + f.qk_rope, 1);
+        CK(cudaGetLastError());
       }
-      CK(cudaMemcpy2DAsync(rows, rowb, (const uint8_t*)k_or_latent + (size_t)l * n_tokens * lat, lat, lat, n_tokens,
-                           cudaMemcpyDefault, c->stream));
-      CK(cudaMemcpy2DAsync(rows + lat, rowb, (const uint8_t*)v_or_pe + (size_t)l * n_tokens * pe, pe, pe, n_tokens,
-                           cudaMemcpyDefault, c->stream));
-      mla_cache_convert<<<1184, 256, 0, c->stream>>>(rows, (uint8_t*)c->kc[l], n_tokens, f.kv_lora + f.qk_rope, 1);
-      CK(cudaGetLastError());
     }
-  }
+    return DEC_OK;
+  };
+  rc = copy_layers();
   if (rows) {
-    CK(cudaStreamSynchronize(c->stream));
-    CK(cudaFree(rows));
+    const cudaError_t es = cudaStreamSynchronize(c->stream);
+    const cudaError_t ef = cudaFree(rows);
+    if (!rc && (es != cudaSuccess || ef != cudaSuccess))
+      return fail(c, DEC_ERR_CUDA, "cache scratch: %s", cudaGetErrorString(es != cudaSuccess ? es : ef));
   }
+  if (rc) return rc;
   StepState st{1, n_tokens, 0, 0};
   CK(cudaMemcpyAsync(c->d_state, &st, sizeof st, cudaMemcpyHostToDevice, c->stream));
   CK(cudaStreamSynchronize(c->stream));

@@ -112,3 +112,29 @@ def test_wrong_weight_size_is_rejected(pkg):
         assert e.value.code == pkg.dec.DEC_ERR_INVALID_ARG
     finally:
         d.close()
+
+
+def test_a_stream_given_to_the_decoder_stays_the_callers(pkg):
+    """dec_set_stream borrows the caller's stream: after dec_destroy the stream still works, and
+    the step it ran gives the same token as a decoder on the library's own stream (bf16 model:
+    the drawn cache is bf16, the layout dec_set_kv_cache takes for it)."""
+    w = workloads.get("small_dense_bf16")
+    k, v = sdev.synthetic_cache_device(w)
+    s = torch.cuda.Stream()
+    d = _decoder(pkg, w)
+    try:
+        d.set_stream(s.cuda_stream)
+        d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        tok = d.step(3)
+    finally:
+        d.close()
+    with torch.cuda.stream(s):
+        y = (torch.arange(1024, device="cuda", dtype=torch.float32) * 2).sum()
+    s.synchronize()
+    assert float(y) == 1024.0 * 1023.0
+    d2 = _decoder(pkg, w)
+    try:
+        d2.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        assert d2.step(3) == tok
+    finally:
+        d2.close()
