@@ -123,3 +123,17 @@ def test_gqa_group_above_eight_is_rejected():
     with pytest.raises(pkg.DecError) as e:
         pkg.Decoder(pkg.config_from_workload(w))
     assert e.value.code == pkg.dec.DEC_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", sorted(__import__("synth.workloads", fromlist=["WORKLOADS"]).WORKLOADS))
+def test_every_named_workload_passes_validation(name):
+    """Each workload's configuration is accepted by the library's checks: without a GPU,
+    dec_create gets as far as its first device call and fails there, not at validation."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    import persistent_sm_decode_02_b200 as pkg
+    from synth import workloads
+    with pytest.raises(pkg.DecError) as e:
+        pkg.Decoder(pkg.config_from_workload(workloads.get(name)))
+    assert e.value.code == pkg.dec.DEC_ERR_CUDA and "cudaSetDevice" in str(e.value)
