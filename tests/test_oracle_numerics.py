@@ -81,6 +81,23 @@ def test_gemv_against_brute_force(dtype):
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
 
 
+def test_fp8_block_dequant_against_scalar_definition():
+    """w[n, k] = E4M3(q[n, k]) * s[n // 128, k // 128] on a ragged 2 x 3 block grid, whose
+    distinct per-block scales expose a transposed or shifted block index."""
+    rng = np.random.default_rng(12)
+    N, K = 200, 300
+    q = rng.integers(0, 256, size=(N, K), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x22
+    s = np.array([[1.0, 2.0, 4.0], [8.0, 16.0, 32.0]], dtype=np.float32)
+    W = nm.dequant_fp8_b128(q, s)
+    assert W.shape == (N, K)
+    for n, k in [(0, 0), (127, 127), (128, 0), (0, 128), (199, 299), (150, 260), (5, 256)]:
+        assert W[n, k] == nm.e4m3_value(int(q[n, k])) * float(s[n // 128, k // 128])
+    ref = np.array([[nm.e4m3_value(int(q[n, k])) * float(s[n // 128, k // 128]) for k in range(K)]
+                    for n in range(0, N, 7)])
+    np.testing.assert_array_equal(W[::7], ref)
+
+
 def test_softmax_brute_force_and_sum():
     x = np.array([0.3, -1.2, 5.0, 5.0, 2.2])
     e = [math.exp(v - 5.0) for v in x]
