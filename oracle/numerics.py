@@ -134,6 +134,7 @@ def topk_lowest_index(p: np.ndarray, k: int) -> np.ndarray:
 
 
 def margin_topk(logits: np.ndarray, k: int) -> float:
-    """Gap between the k-th and (k+1)-th largest entries (0 if fewer than k+1 entries)."""
+    """Gap between the k-th and (k+1)-th largest entries; infinite when there is no (k+1)-th
+    entry (the top-k set is then forced, so no decision is near a tie)."""
     s = np.sort(np.asarray(logits, dtype=np.float64))[::-1]
     return float(s[k - 1] - s[k]) if s.shape[0] > k else float("inf")

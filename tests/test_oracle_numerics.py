@@ -158,6 +158,14 @@ def test_topk_matches_full_sort_with_ties():
         assert np.array_equal(idx, ref)
 
 
+def test_margin_topk_hand_example():
+    x = np.array([3.0, 1.0, 2.0, 2.0])
+    assert nm.margin_topk(x, 1) == 1.0          # 3 vs 2
+    assert nm.margin_topk(x, 2) == 0.0          # the two 2s tie across the cut
+    assert nm.margin_topk(x, 3) == 1.0          # 2 vs 1
+    assert nm.margin_topk(x, 4) == float("inf")  # nothing outside the set
+
+
 def test_route_weights_sum_to_one():
     rng = np.random.default_rng(9)
     for k in (1, 4, 8):
