@@ -71,3 +71,11 @@ def test_peak_fallback_without_measured_file(monkeypatch, tmp_path):
     assert bench.measured_peaks() == (6650.0, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6450.5}))
     assert bench.measured_peaks() == (6450.5, "measured")
+
+
+def test_l2_note_tells_streaming_from_warm_steps():
+    from synth import workloads as wl
+    big = wl.active_bytes_per_token(wl.get("moe_mla_fp8_1k"), 1024)["total"]
+    tiny = wl.active_bytes_per_token(wl.get("tiny_dense_f32"), 64)["total"]
+    assert "far above" in bench.l2_note(big)
+    assert "warm" in bench.l2_note(tiny) and "far above" not in bench.l2_note(tiny)
