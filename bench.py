@@ -60,9 +60,9 @@ def recorded_traffic(workload: str):
         return None
     with open(p) as f:
         d = json.load(f)
-    # A record stays valid across later source changes that it lists as host-only (the kernel,
-    # the task plan and the launch are the ones that were captured).
-    valid = {d.get("source_hash")} | {x["source_hash"] for x in d.get("host_only_changes", [])}
+    # A record stays valid across the later source states it lists as leaving the kernel, the
+    # task plan and the launch as captured (host-only or comment-only changes).
+    valid = {d.get("source_hash")} | {x["source_hash"] for x in d.get("same_kernel_sources", [])}
     if source_hash() not in valid:
         return None
     return d.get("dram_bytes_per_step")

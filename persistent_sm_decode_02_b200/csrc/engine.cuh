@@ -9,7 +9,7 @@
 //     the consumers wait for the previous layer; only routed-expert weights
 //     wait, because their address comes from the router's top-k;
 //   * 1 signaller warp publishes each finished task: it receives the task from
-//     the consumers through a two-slot mailbox guarded by mbarriers and does
+//     the consumers through a 16-slot mailbox guarded by mbarriers and does
 //     the gpu-scope fence and counter release, off the consumers' path.
 // Consumers wait on the dependency counters of the task's op (one thread polls,
 // then a barrier), build the task's input vector in shared memory (norm /
@@ -710,7 +710,7 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
 
 // MLA: the step's new latent cache row, c = bf16(RMSNorm(kv_a latent) * g) and
 // k_pe = bf16(RoPE(kv_a rope part)), stored at position pos of the blocked cache
-// (all consumer threads; absorb_q's first task, before attention reads the block).
+// (all consumer threads; absorb_q's extra last task, before attention reads the block).
 __device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
   Misc* m = S.m;
   const int tid = threadIdx.x, pos = m->st.pos;
@@ -1141,13 +1141,13 @@ __device__ __forceinline__ void attn_consume(const KParams& P, const OpDesc& od,
 //   S = Q . C^T : Q = [q_lat | q_pe] bf16 [128 x (kvl + rdim)], C = the block's
 //                 cache rows [64 x (kvl + rdim)]; nine 64-dim K-chunks, each
 //                 ring stage carrying Q's chunk (16 KB) and C's chunk (8 KB).
-//   P = exp(S * scale - m) per head (one thread per head reads its TMEM row),
+//   P = exp(S * scale - m) per head (8 warps, each 32 heads x 32 positions of TMEM),
 //       split into bf16 hi + lo parts so that P keeps ~16 mantissa bits.
 //   O = P . C_lat : two ring stages of 256 latent dims (32 KB each); C is
 //                 read MN-major from the same bytes the S step read K-major.
 // The task publishes (m, l, O) for the split-KV log-sum-exp combine in the uv
 // projection's prologue.  The step's new latent row is already in the cache:
-// absorb_q's first task writes it (mla_new_row).
+// absorb_q's extra last task writes it (mla_new_row).
 // TMEM: 512 fp32 columns x 128 lanes; S uses columns 0..63 and is read out
 // before O (columns 0..511) overwrites it.
 __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S, uint32_t& g,

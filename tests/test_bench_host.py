@@ -58,7 +58,7 @@ def test_recorded_traffic_needs_the_matching_source(monkeypatch):
         d = json.load(f)
     monkeypatch.setattr(bench, "source_hash", lambda: d["source_hash"])
     assert bench.recorded_traffic(d["workload"]) == d["dram_bytes_per_step"]
-    for x in d.get("host_only_changes", []):
+    for x in d.get("same_kernel_sources", []):
         monkeypatch.setattr(bench, "source_hash", lambda: x["source_hash"])
         assert bench.recorded_traffic(d["workload"]) == d["dram_bytes_per_step"]
     monkeypatch.setattr(bench, "source_hash", lambda: "0" * 16)
