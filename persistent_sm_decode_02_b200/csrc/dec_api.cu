@@ -582,7 +582,7 @@ static int build_plan(dec_ctx* c) {
         o.rdim = rd;
         o.rope_cos = c->rope_cos;
         o.rope_sin = c->rope_sin;
-        // its first task also appends the step's latent row (normalised c, RoPE'd k_pe) to the cache
+        // an extra last task appends the step's latent row (normalised c, RoPE'd k_pe) to the cache
         const OpDesc& p1 = c->ops[s1];
         o.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
         o.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
@@ -980,9 +980,9 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
     for (auto& o : c->ops)
       if (o.router) o.route_dump = c->d_route_dump + f.top_k * i++;
   }
-  // per op: the dependency counter, then (routers) the finished-task counter
-  // per op: the dependency counter and the router's finished-task counter; per dense
-  // attention op: one finished-task counter per kv head. All reset together.
+  // Counters, one array that dec_reset zeroes: per op the dependency counter and
+  // (routers) the finished-task counter, the latter at ops.size() + op; per dense
+  // attention op one finished-task counter per kv head, after those.
   c->n_counters = 2 * c->ops.size();
   for (auto& o : c->ops)
     if (o.kind == OP_ATTN) c->n_counters += o.hkv;
