@@ -46,6 +46,8 @@ extern "C" {
 #define DEC_ERR_CUDA (-5)        /* a CUDA runtime call failed */
 #define DEC_ERR_TIMEOUT (-6)     /* a device-side wait gave up; context poisoned until dec_reset */
 #define DEC_ERR_UNSUPPORTED (-7) /* configuration outside what the kernels implement */
+#define DEC_ERR_NUMERIC (-8)     /* a router or LM-head logit was NaN or infinite (corrupt weights or
+                                    activations); context poisoned until dec_reset */
 
 /* ------------------------------------------------------------------ enums */
 #define DEC_ARCH_DENSE 0   /* RMSNorm, GQA attention with RoPE, SwiGLU FFN */
@@ -98,15 +100,20 @@ enum {
 /* dec_debug_dump selectors */
 #define DEC_DUMP_KV 1       /* dense: K then V, [n_layers][n_kv_heads][len][head_dim]; MLA: latent then pe */
 #define DEC_DUMP_ROUTES 2   /* MoE: int32 [n_moe_layers][top_k] expert ids of the last step */
-#define DEC_DUMP_TRACE 3    /* uint64 records {cta<<48|op<<32|task, t_start, t_first_stage, t_done, t_published}
-                               (ns, %globaltimer) of every task of the last step */
-#define DEC_DUMP_TRACE_PRODUCER 6 /* uint64 pairs {cta<<48|op<<32|task, t_reached} per task-list position: when the
-                                     weight-streaming warp reached each task (ns) */
+#define DEC_DUMP_TRACE 3    /* uint64 records {cta<<48|op<<32|task, t_start, t_input_ready, t_first_stage, t_done,
+                               t_published} (ns, %globaltimer) of every task of the last step */
+#define DEC_DUMP_TRACE_PRODUCER 6 /* uint64 triples {cta<<48|op<<32|task, t_reached, t_first_issued} per task-list
+                                     position: when the weight-streaming warp reached each task and issued its
+                                     first stage (ns; 0 for a task that streams nothing) */
 #define DEC_DUMP_PLAN 4     /* text: one line per op (kind, tasks, geometry) */
 #define DEC_DUMP_WEIGHTS 5  /* bytes of weights read per step (uint64 x2: weights+scales, stored incl. padding) */
+#define DEC_DUMP_STATUS 7   /* int32 x12: device status word {code, cta, op, task} (code 0 ok, 1 timeout,
+                               2 non-finite logit), then the step state {epoch, pos, tok, last, stop, 0, 0, 0} */
 #define DEC_DUMP_OP 100     /* + op index (DEC_DUMP_PLAN order): fp32 outputs of that op in the last step;
-                               GEMV ops: partial sums [splits][rows]; attention ops: max [heads][chunks],
-                               sum [heads][chunks], weighted values [heads][chunks][dim], concatenated */
+                               GEMV ops: [rows] (ops whose rows add into one accumulator, the routed and
+                               shared experts' down projections, give the same summed vector); attention
+                               ops: max [heads][chunks], sum [heads][chunks], weighted values
+                               [heads][chunks][dim], concatenated */
 
 /* ------------------------------------------------------------------ types */
 typedef struct dec_ctx dec_ctx; /* opaque; owns all of its device memory */
@@ -142,19 +149,27 @@ typedef struct dec_tensor {
 
 /* Validate the configuration, plan the task list of one decode step and
  * allocate all device memory (weights, caches, activations, counters).
+ * Defined by: TileRT 是什么 §六 6.1 (the "prepare money" call that sets up each
+ * GPU's parameters and buffers) and §六 6.2 (operator decomposition, execution
+ * planning and memory layout done once, at compile time, not per step).
  * On an error *out may still hold a context that carries the message for
  * dec_last_error; pass it to dec_destroy, which frees what was allocated.
  * Errors: INVALID_ARG (bad config), UNSUPPORTED, OOM, CUDA. */
 int dec_create(const dec_config* cfg, dec_ctx** out);
 
 /* Copy n weight tensors into the context, re-laid out into its tile order
- * (host-to-device or device-to-device).  May be called repeatedly; a step
+ * (host-to-device or device-to-device).  Defined by: TileRT 是什么 §六 6.2
+ * (weight preprocessing belongs to compile time) and §五 5.3 (each GPU manages
+ * its own parameters).  May be called repeatedly; a step
  * requires every tensor of the model to have been loaded once.
  * Errors: INVALID_ARG (unknown kind, bad layer/expert, size mismatch), CUDA. */
 int dec_load_weights(dec_ctx* c, const dec_tensor* t, int n);
 
 /* Install a prefilled context of n_tokens positions (the KV cache another
- * engine produced) and set the decode position to n_tokens.
+ * engine produced) and set the decode position to n_tokens.  Defined by: the
+ * InferenceX article's PD-disaggregation section (prefill runs in another
+ * engine, which moves its KV cache to the decode node) and TileRT 是什么 §五 5.3
+ * (the kv_cache and pe_cache buffers of MLA).
  * Dense: k, v as [n_layers][n_kv_heads][n_tokens][head_dim].
  * MLA:   latent [n_layers][n_tokens][kv_lora] (the kv_cache) and
  *        pe [n_layers][n_tokens][qk_rope] (the pe_cache).
@@ -163,31 +178,69 @@ int dec_load_weights(dec_ctx* c, const dec_tensor* t, int n);
  * Errors: INVALID_ARG, CAPACITY (n_tokens >= max_seq), CUDA. */
 int dec_set_kv_cache(dec_ctx* c, const void* k_or_latent, const void* v_or_pe, int32_t n_tokens);
 
-/* One decode step, synchronous: embed token_id at the current position,
+/* One decode step, synchronous (TileRT 是什么 §六 6.1, the "show hands" inference
+ * call; InferenceX article, "what TileRT is": the step as one persistent kernel
+ * of overlapped tile tasks): embed token_id at the current position,
  * run every layer, write the fp32 logits [vocab] to out_logits (nullable;
  * host or device) and the greedy token (argmax, lowest id on ties) to
  * *out_next_token (host, nullable).  token_id < 0 feeds back the previous
  * step's greedy token from device memory.
  * Errors: STATE (weights or context missing, or poisoned), CAPACITY,
- * INVALID_ARG (token_id >= vocab), TIMEOUT, CUDA. */
+ * INVALID_ARG (token_id >= vocab), TIMEOUT, NUMERIC, CUDA. */
 int dec_step(dec_ctx* c, int32_t token_id, float* out_logits, int32_t* out_next_token);
 
 /* Enqueue one decode step on the context's stream and return at once.
  * token_id < 0 feeds back the previous step's greedy token on the device, so
  * steps chain without host round trips.  Logits stay in the context.
- * Errors as dec_step except TIMEOUT, which dec_sync reports. */
+ * Errors as dec_step except TIMEOUT and NUMERIC, which dec_sync reports. */
 int dec_step_async(dec_ctx* c, int32_t token_id);
 
 /* Wait for enqueued steps; copy the last greedy token to *out_next_token
  * (nullable) and the last logits to out_logits (nullable, host or device).
- * Errors: TIMEOUT (context poisoned), CUDA. */
+ * Errors: TIMEOUT or NUMERIC (context poisoned), CUDA. */
 int dec_sync(dec_ctx* c, float* out_logits, int32_t* out_next_token);
 
+/* Generation: a whole decode lifetime with the host out of the loop (InferenceX
+ * article, "what TileRT is": the host launches the engine kernel once and the
+ * decode stays on the GPU).  token_id (< 0: the previous step's greedy token) is
+ * embedded at the current position; each step's greedy token is fed back on the
+ * device.  In DEC_PERSISTENT mode ONE kernel launch runs all steps and writes every
+ * greedy token into a host-mapped ring as soon as it is known; in DEC_PER_OP and
+ * DEC_PER_OP_GRAPH modes the same steps run one launch per step with a host check
+ * after each (the ablation).  The generation ends after n_steps steps, after the
+ * step whose greedy token equals stop_token (-1: none), or after the step during
+ * which dec_generate_stop was called.  While it runs, every call that would queue
+ * work or change the context returns DEC_ERR_STATE; dec_generate_poll and
+ * dec_generate_stop may be called from the same host thread at any time.
+ * Errors: STATE, CAPACITY (position + n_steps > max_seq), INVALID_ARG, CUDA. */
+int dec_generate_async(dec_ctx* c, int32_t token_id, int32_t n_steps, int32_t stop_token);
+
+/* Tokens of the running generation produced so far, without waiting: copies
+ * min(count, cap) tokens into out_tokens (host), *out_count = count (nullable),
+ * *out_done = 1 once the generation's launches have finished (nullable).
+ * Errors: STATE (no generation), INVALID_ARG, CUDA. */
+int dec_generate_poll(dec_ctx* c, int32_t* out_tokens, int32_t cap, int32_t* out_count, int32_t* out_done);
+
+/* Ask the running generation to end after the step in progress (a host-mapped
+ * flag the final op of every step reads).  Returns at once. */
+int dec_generate_stop(dec_ctx* c);
+
+/* Wait for the generation to finish; copy its tokens (at most cap) to out_tokens
+ * (host) and their number to *out_count (nullable).  The position advances by the
+ * steps completed.  Errors: TIMEOUT or NUMERIC (context poisoned), STATE, CUDA. */
+int dec_generate_wait(dec_ctx* c, int32_t* out_tokens, int32_t cap, int32_t* out_count);
+
+/* dec_generate_async then dec_generate_wait (out_tokens holds n_steps entries). */
+int dec_generate(dec_ctx* c, int32_t token_id, int32_t n_steps, int32_t stop_token, int32_t* out_tokens,
+                 int32_t* out_count);
+
 /* Forget the context (position 0), clear a poisoned state, re-zero the
- * dependency counters.  Weights are kept. */
+ * dependency counters.  Weights are kept.  Defined by: TileRT 是什么 §六 6.1 (the
+ * reset call that starts a new sequence). */
 int dec_reset(dec_ctx* c);
 
-/* Free everything the context owns.  Accepts NULL. */
+/* Free everything the context owns.  Accepts NULL.  Defined by: TileRT 是什么
+ * §六 6.1 (the "go home" call that releases the resources). */
 int dec_destroy(dec_ctx* c);
 
 /* Use `stream` (a cudaStream_t, NULL = the legacy default stream) for all
@@ -226,22 +279,29 @@ const char* dec_last_error(const dec_ctx* c);
  * split into position chunks whose (max, sum, weighted values) are combined
  * with a log-sum-exp rescale -- the same split-KV attention the decode step
  * runs.
- *   q        device, fp32 [n_heads][head_dim] (already RoPE'd and rounded as wanted)
- *   k_cache  device, bf16 [n_kv_heads][cache_stride][head_dim]
- *   v_cache  device, bf16 [n_kv_heads][cache_stride][head_dim]
- *   out      device, fp32 [n_heads][head_dim]
+ *   q        device, fp32 [n_heads][head_dim] (already RoPE'd and rounded as wanted), 4-byte aligned
+ *   k_cache  device, bf16 [n_kv_heads][cache_stride][head_dim], 16-byte aligned
+ *   v_cache  device, bf16 [n_kv_heads][cache_stride][head_dim], 16-byte aligned
+ *   out      device, fp32 [n_heads][head_dim], 4-byte aligned
  *   stream   cudaStream_t (NULL = legacy default stream); the call is asynchronous.
+ * A pointer that breaks its alignment returns INVALID_ARG before anything runs.
  * Limits: head_dim 64 or 128, n_heads a multiple of n_kv_heads with at most 8
  * query heads per kv head, 1 <= n_pos <= cache_stride, and the per-chunk
  * partials n_heads * chunks * (head_dim + 2) floats must fit the library's
- * fixed 2 MiB scratch (the call uses fewer chunks when needed and returns
- * DEC_ERR_CAPACITY if even one chunk per head does not fit).
+ * fixed 2 MiB scratch.  The call takes about 148 / n_kv_heads chunks per kv head
+ * (1 to 64, at most n_pos), which stays far inside the scratch while n_kv_heads
+ * <= 148; it returns DEC_ERR_CAPACITY when even one chunk per head does not fit
+ * (n_heads * (head_dim + 2) > 524288).
  * The scratch is a fixed array inside the library, held by every GPU that
  * loads it until the process exits, and shared by all calls: nothing in it has
  * to start at zero (every call writes what it reads), but calls whose kernels
  * overlap on the GPU (for example on two streams) race on it.  The first call
  * on each device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before any stream capture.
+ * make that first call before any stream capture.  The address is kept for
+ * the life of the process: after cudaDeviceReset (or any other teardown of the
+ * device's primary context) this function must not be called again.
+ * If a CUDA error from an earlier runtime call of this library is still
+ * pending, the call returns CUDA without launching and leaves it pending.
  * Errors: INVALID_ARG, CAPACITY, CUDA.  No context, no dec_last_error. */
 int dec_attention_noalloc(const float* q, const void* k_cache, const void* v_cache, int32_t n_heads,
                           int32_t n_kv_heads, int32_t head_dim, int32_t n_pos, int32_t cache_stride, float* out,

@@ -271,6 +271,22 @@ def route_topk(router_logits: np.ndarray, k: int):
     return idx, wts
 
 
+def mla_absorb_query(qn, W_UK):
+    """q_lat^h = W_UK^h^T q_nope^h: the query mapped into the latent space (qn [H, nope], W_UK [H, nope, kv_lora])."""
+    return np.einsum("hjc,hj->hc", W_UK, qn)
+
+
+def mla_latent_attention(q_lat, qpe, C, PE, scale):
+    """s_h(t) = (q_lat^h . c_t + q_pe^h . kpe_t) * scale; O_lat^h = sum_t softmax(s_h)_t c_t."""
+    s = (q_lat @ C.T + qpe @ PE.T) * scale
+    return softmax(s, axis=1) @ C
+
+
+def mla_up_value(O_lat, W_UV):
+    """o^h = W_UV^h O_lat^h (O_lat [H, kv_lora], W_UV [H, v, kv_lora])."""
+    return np.einsum("hvc,hc->hv", W_UV, O_lat)
+
+
 def mla_absorbed(qn, qpe, C, PE, W_UK, W_UV, R=identity):
     """Absorbed MLA for one token: q_lat^h = W_UK^h^T q_nope^h; s_h(t) = (q_lat^h . c_t + q_pe^h . kpe_t)
     / sqrt(d_nope + d_rope); O_lat^h = sum_t softmax(s_h)_t c_t; o^h = W_UV^h O_lat^h.
@@ -278,10 +294,9 @@ def mla_absorbed(qn, qpe, C, PE, W_UK, W_UV, R=identity):
     qn [H, nope], qpe [H, rope], C [T, kv_lora], PE [T, rope], W_UK [H, nope, kv_lora], W_UV [H, v, kv_lora].
     """
     scale = 1.0 / math.sqrt(qn.shape[1] + qpe.shape[1])
-    q_lat = R(np.einsum("hjc,hj->hc", W_UK, qn))
-    s = (q_lat @ C.T + qpe @ PE.T) * scale
-    O_lat = softmax(s, axis=1) @ C
-    return np.einsum("hvc,hc->hv", W_UV, R(O_lat))
+    q_lat = R(mla_absorb_query(qn, W_UK))
+    O_lat = mla_latent_attention(q_lat, qpe, C, PE, scale)
+    return mla_up_value(R(O_lat), W_UV)
 
 
 def mla_unabsorbed(qn, qpe, C, PE, W_UK, W_UV):

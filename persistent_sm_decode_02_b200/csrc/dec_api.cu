@@ -32,7 +32,7 @@ namespace {
 // A weight matrix stored in tile order: [row tile][split][stage][R][kcb bytes].
 struct Mat {
   int N = 0, K = 0, wb = 1, wtype = WT_F32;
-  int R = 0, S = 1, nst = 1, kcb = 0, Kpad = 0, ntiles = 0;
+  int R = 0, nst = 1, kcb = 0, Kpad = 0, ntiles = 0;  // nst: stages per row tile
   int n_experts = 1;
   int mode = 0;  // source layout: 0 row-major [N][K]; 1 W_UK^T of kv_b; 2 W_UV of kv_b
   size_t tile_bytes = 0;  // bytes of one expert
@@ -58,9 +58,9 @@ Geo gemv_geometry(int K, int wb) {
   int best = -1;
   long long best_waste = 1LL << 62;
   // Prefer 512-byte row chunks: 32 lanes cover a row, so every row reduces
-  // inside one warp and tasks need no CTA-wide barrier; wider chunks only when
+  // inside one warp and tasks need no CTA-wide barrier; narrower chunks only when
   // 512 would pad K too much.
-  for (int kcb = 512; kcb >= 32; kcb >>= 1) {
+  for (int kcb = 512; kcb >= 64; kcb >>= 1) {  // the widths the kernels are compiled for
     const long long pad = (Kb + kcb - 1) / kcb * kcb;
     const long long waste = pad - Kb;
     if (waste * 16 <= Kb) {
@@ -83,32 +83,9 @@ Geo gemv_geometry(int K, int wb) {
   return g;
 }
 
-// Split-K factor S of a GEMV op, in units of ring stages on the busiest CTA: its tasks'
-// stages plus a fixed cost per task, plus the consumer's prologue, which reads all S
-// partial vectors (out_rows fp32 values each) on every CTA.  Every CTA reads the same lines
-// at once, and that L2 read ran about 4x slower per byte than a weight stage in the device
-// trace, hence the weight.
-constexpr double kPrologueWeight = 4.0;
-int choose_split(int ntiles, int nst_total, int n_ctas, long long out_rows, bool force_one) {
-  if (force_one) return 1;
-  int best = 1;
-  double best_cost = 1e30;
-  for (int S = 1; S <= 16 && S <= nst_total; ++S) {
-    if (nst_total % S) continue;
-    const long long tasks = (long long)ntiles * S;
-    const long long per = (tasks + n_ctas - 1) / n_ctas;
-    const double cost = per * (nst_total / (double)S + 0.75) + kPrologueWeight * S * out_rows * 4.0 / kStageBytes;
-    if (cost < best_cost - 1e-9) {
-      best_cost = cost;
-      best = S;
-    }
-  }
-  return best;
-}
-
-__global__ void relayout16(const uint8_t* src, long long N, long long K, int wb, int R, int S, int nst, int kcb,
+__global__ void relayout16(const uint8_t* src, long long N, long long K, int wb, int R, int nst, int kcb,
                            long long total16, uint8_t* dst) {
-  // dst byte q = ((((rt*S + s)*nst + st)*R + r)*kcb + jb); one thread per 16 bytes
+  // dst byte q = (((rt*nst + st)*R + r)*kcb + jb); one thread per 16 bytes
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total16;
        i += (long long)gridDim.x * blockDim.x) {
     const long long q = i * 16;
@@ -117,11 +94,9 @@ __global__ void relayout16(const uint8_t* src, long long N, long long K, int wb,
     const long long r = rest % R;
     rest /= R;
     const long long st = rest % nst;
-    rest /= nst;
-    const long long s = rest % S;
-    const long long rt = rest / S;
+    const long long rt = rest / nst;
     const long long n = rt * R + r;
-    const long long kb = (s * nst + st) * kcb + jb;  // byte offset in the padded row
+    const long long kb = st * kcb + jb;  // byte offset in the padded row
     uint4 v = make_uint4(0, 0, 0, 0);
     if (n < N && kb < K * wb) v = *reinterpret_cast<const uint4*>(src + n * K * wb + kb);
     *reinterpret_cast<uint4*>(dst + q) = v;
@@ -129,7 +104,7 @@ __global__ void relayout16(const uint8_t* src, long long N, long long K, int wb,
 }
 
 // Element-wise re-layout for the two views of kv_b (mode 1: W_UK^T, mode 2: W_UV).
-__global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long long K, int wb, int R, int S, int nst,
+__global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long long K, int wb, int R, int nst,
                              int kcb, long long total, int nope, int vdim, int kvl, uint8_t* dst) {
   for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < total;
        q += (long long)gridDim.x * blockDim.x) {
@@ -138,11 +113,9 @@ __global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long lon
     const long long r = rest % R;
     rest /= R;
     const long long st = rest % nst;
-    rest /= nst;
-    const long long s = rest % S;
-    const long long rt = rest / S;
+    const long long rt = rest / nst;
     const long long n = rt * R + r;
-    const long long kb = (s * nst + st) * kcb + jb;
+    const long long kb = st * kcb + jb;
     const long long k = kb / wb, byte = kb % wb;
     uint8_t v = 0;
     if (n < N && k < K) {
@@ -200,9 +173,6 @@ struct dec_ctx {
   std::vector<OpDesc> ops;
   std::vector<std::string> op_names;
   OpDesc* d_ops = nullptr;
-  int2* d_tasks = nullptr;
-  int* d_task_off = nullptr;
-  std::vector<int> task_off;
   int lm_op = -1, final_op = -1;
   // memory
   std::vector<void*> allocs;
@@ -235,12 +205,26 @@ struct dec_ctx {
   cudaGraphExec_t graph = nullptr;
   int mode = DEC_PERSISTENT;
   std::vector<std::vector<void*>> seg_mats;  // per op: the Mat behind every segment
+  unsigned* d_cursors = nullptr;             // task cursors [2][n_cursors]
+  int n_cursors = 0;
+  std::vector<std::pair<void*, size_t>> accs;  // fixed-point accumulators, cleared by dec_reset
   uint8_t* staging = nullptr;
   size_t staging_bytes = 0;
   void* kvb_src = nullptr;
   const void* kernel = nullptr;  // engine instance for this model's weight type and attention kind
   size_t weight_bytes_step = 0, weight_bytes_stored = 0;
+  // generation (dec_generate*): host-mapped token ring, count and stop word
+  GenState* d_gen = nullptr;
+  uint8_t* h_map = nullptr;  // [count u32 | stop i32 | pad | ring i32[max_seq]]
+  uint8_t* d_map = nullptr;
+  bool generating = false;
+  int gen_epoch0 = 0, gen_steps = 0, gen_stop_token = -1;
+  cudaEvent_t gen_done = nullptr;
 };
+
+static volatile unsigned* h_count(dec_ctx* c) { return reinterpret_cast<volatile unsigned*>(c->h_map); }
+static volatile int* h_stop(dec_ctx* c) { return reinterpret_cast<volatile int*>(c->h_map + 4); }
+static volatile int* h_ring(dec_ctx* c) { return reinterpret_cast<volatile int*>(c->h_map + 16); }
 
 static int fail(dec_ctx* c, int code, const char* fmt, ...) __attribute__((format(printf, 3, 4)));
 static int fail(dec_ctx* c, int code, const char* fmt, ...) {
@@ -296,6 +280,7 @@ struct Planner {
     o.layer = layer;
     o.dep[0] = o.dep[1] = -1;
     o.pdep = -1;
+    o.ngroups = 1;
     o.in_bf16 = c->act_bf16;
     o.eps = c->cfg.norm_eps;
     return o;
@@ -313,18 +298,18 @@ struct Planner {
   }
 
   // Create a GEMV op over segments sharing K; returns op index.
-  // whole_reader: every CTA running the consumer reads the whole output (a GEMV prologue);
-  // false when each consumer task reads only its own slice (attention reading q/k/v).
-  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool force_s1, const char* name,
-           bool whole_reader = true) {
+  // A row tile of more than kPieceStages ring stages is cut along K into equal pieces
+  // (one task each) that add into a fixed-point accumulator (dec_types.h), so tasks
+  // stay short and the run-time task hand-out can balance the SMs; whole_tiles keeps
+  // one task per tile with an fp32 output row (the LM head's argmax keys, absorb_q's
+  // bf16 query, ops grouped per head).  same_rows: every segment adds into the same
+  // output rows (the experts' down projections, the routed ones weighted by the router),
+  // which also needs the accumulator.  Segments that read different input groups get
+  // one task cursor each.
+  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool whole_tiles, const char* name,
+           bool same_rows = false, bool fp32_out = false) {
     OpDesc o = base_op(OP_GEMV, layer);
     const Geo g = gemv_geometry(K, c->wb);
-    int ntiles = 0;
-    for (auto& s : segs) ntiles += (s.mat->N + g.R - 1) / g.R;
-    long long out_rows = 0;
-    if (whole_reader)
-      for (auto& sp : segs) out_rows += sp.mat->N;
-    const int S = choose_split(ntiles, g.nst_total, c->n_ctas, out_rows, force_s1);
     o.wtype = c->wtype;
     o.K = K;
     o.Kpad = g.Kpad;
@@ -334,24 +319,28 @@ struct Planner {
     o.G = g.G;
     o.rpt = g.rpt;
     o.R = g.R;
-    o.S = S;
-    o.nst = g.nst_total / S;
+    o.nst_total = g.nst_total;
     o.n = K;
     o.nsegs = (int)segs.size();
     if (o.nsegs > kMaxSegs) {
       rc = fail(c, DEC_ERR_UNSUPPORTED, "too many segments in %s", name);
       return -1;
     }
+    const int nps = whole_tiles ? 1 : (g.nst_total + kPieceStages - 1) / kPieceStages;  // pieces per tile
+    const bool acc = nps > 1 || same_rows;  // tasks add into rows (else one task stores each row)
+    bool groups = false;
+    for (auto& sp : segs) groups |= sp.in_group != segs[0].in_group;
     int task = 0, out = 0;
+    std::vector<int4> pieces;
+    std::vector<int> gb;
     for (int i = 0; i < o.nsegs; ++i) {
       Mat* m = segs[i].mat;
       m->R = g.R;
-      m->S = S;
-      m->nst = o.nst;
+      m->nst = g.nst_total;
       m->kcb = g.kcb;
       m->Kpad = g.Kpad;
       m->ntiles = (m->N + g.R - 1) / g.R;
-      m->tile_bytes = (size_t)m->ntiles * S * o.nst * g.R * g.kcb;
+      m->tile_bytes = (size_t)m->ntiles * g.nst_total * g.R * g.kcb;
       m->sc_count = c->wtype == WT_FP8 ? (size_t)((m->N + 127) / 128) * ((m->K + 127) / 128) : 0;
       Seg& sg = o.seg[i];
       sg.slot = segs[i].slot;
@@ -359,15 +348,48 @@ struct Planner {
       sg.N = m->N;
       sg.ntiles = m->ntiles;
       sg.task0 = task;
-      sg.out_off = out;
+      sg.out_off = same_rows ? 0 : out;
       sg.w_estride = (long long)m->tile_bytes;
       sg.s_estride = (long long)m->sc_count;
-      task += m->ntiles * S;
-      out += m->N;
+      sg.zero_acc = acc && (!same_rows || i == 0);
+      if (groups) gb.push_back(acc ? (int)pieces.size() : task);
+      if (acc)
+        for (int r = 0; r < m->ntiles; ++r)
+          for (int p = 0; p < nps; ++p) {
+            const int a = p * g.nst_total / nps, b = (p + 1) * g.nst_total / nps;
+            pieces.push_back(make_int4(i, r, a, b - a));
+          }
+      task += m->ntiles;
+      if (!same_rows || i == 0) out += m->N;
     }
-    o.ntasks = task;
     o.out_stride = out;
-    int arc = dalloc(c, &o.out, (size_t)o.S * o.out_stride * 4);
+    int arc = DEC_OK;
+    if (fp32_out) {
+      arc = dalloc(c, &o.out, (size_t)o.out_stride * 4);
+    } else if (!(arc = dalloc(c, &o.acc, (size_t)2 * o.out_stride * 8))) {
+      c->accs.push_back({o.acc, (size_t)2 * o.out_stride * 8});
+      o.acc_add = acc ? 1 : 0;
+    }
+    if (arc) {
+    } else if (!acc) {
+      o.ntasks = task;
+    } else {
+      o.ntasks = (int)pieces.size();
+      int4* dp = nullptr;
+      if (!(arc = dalloc(c, &dp, pieces.size() * sizeof(int4))) &&
+          cudaMemcpy(dp, pieces.data(), pieces.size() * sizeof(int4), cudaMemcpyHostToDevice) != cudaSuccess)
+        arc = fail(c, DEC_ERR_CUDA, "piece table of %s", name);
+      o.pieces = dp;
+    }
+    if (!arc && groups) {
+      gb.push_back(o.ntasks);
+      o.ngroups = (int)gb.size() - 1;
+      int* dg = nullptr;
+      if (!(arc = dalloc(c, &dg, gb.size() * sizeof(int))) &&
+          cudaMemcpy(dg, gb.data(), gb.size() * sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        arc = fail(c, DEC_ERR_CUDA, "task groups of %s", name);
+      o.gbegin = dg;
+    }
     if (arc) {
       rc = arc;
       return -1;
@@ -412,7 +434,7 @@ static size_t mla_cache_bytes(const dec_config& f) {
 // Grouped GEMVs whose row tiles are tiny (absorb_q: 16 KB, uv: 32 KB per tile) run a whole
 // input group (one head) per task: the prologue and the task overhead are paid once per head.
 static void group_tasks(OpDesc& o) {
-  if (o.kind != OP_GEMV || o.S != 1 || o.rows_per_group <= 0 || o.rows_per_group % o.R) return;
+  if (o.kind != OP_GEMV || o.pieces || o.rows_per_group <= 0 || o.rows_per_group % o.R) return;
   const int tpt = o.rows_per_group / o.R;
   if (tpt <= 1 || o.ntasks % tpt) return;
   for (int i = 0; i < o.nsegs; ++i)
@@ -423,6 +445,9 @@ static void group_tasks(OpDesc& o) {
 
 static float* gainp(dec_ctx* c, int kind, int layer) { return c->vecs[{kind, layer}].p; }
 
+// The output of GEMV op o from element `off` on, as its consumers read it.
+static PSet out_of(const OpDesc& o, int off = 0) { return PSet{o.acc, o.out_stride, off}; }
+
 static int build_plan(dec_ctx* c) {
   const dec_config& f = c->cfg;
   Planner P{c};
@@ -431,9 +456,8 @@ static int build_plan(dec_ctx* c) {
   const bool mla = f.arch == DEC_ARCH_MLA_MOE;
   // per-layer bookkeeping of the ops whose outputs feed the next layer's residual
   struct LayerOut {
-    int ffn_op = -1;        // dense down op or MoE expert-down op
-    int router_op = -1;     // MoE router op
-    int mid_buf = -1;
+    int ffn_op = -1;   // dense down op, or the MoE layer's routed expert-down op
+    int ffn_op2 = -1;  // MoE: the shared expert's down op (adds into the same accumulator)
   };
   std::vector<LayerOut> lo(L);
   std::vector<float*> h_in(L), h_mid(L);
@@ -454,22 +478,10 @@ static int build_plan(dec_ctx* c) {
       o.embed_bf16 = c->act_bf16;
     } else {
       const LayerOut& p = lo[l - 1];
-      const OpDesc& fo = c->ops[p.ffn_op];
       o.h_base = h_mid[l - 1];
-      if (p.router_op < 0) {
-        o.add = PSet{fo.out, fo.S, fo.out_stride, 0};
-        o.dep[0] = p.ffn_op;
-      } else {
-        const OpDesc& ro = c->ops[p.router_op];
-        o.routed = PSet{fo.out, fo.S, fo.out_stride, 0};
-        o.routed_slot_stride = d;
-        o.rt_w = ro.rt_w;
-        o.n_experts = f.n_experts;
-        o.top_k = f.top_k;
-        if (f.n_shared > 0) o.add2 = PSet{fo.out, fo.S, fo.out_stride, f.top_k * d};
-        o.dep[0] = p.ffn_op;
-        o.dep[1] = p.router_op;
-      }
+      o.add = out_of(c->ops[p.ffn_op]);
+      o.dep[0] = p.ffn_op;
+      o.dep[1] = p.ffn_op2;
     }
   };
 
@@ -489,7 +501,7 @@ static int build_plan(dec_ctx* c) {
       Mat* wq = P.new_mat(DEC_W_Q, l, hq * hd, d, 1, 0);
       Mat* wk = P.new_mat(DEC_W_K, l, hkv * hd, d, 1, 0);
       Mat* wv = P.new_mat(DEC_W_V, l, hkv * hd, d, 1, 0);
-      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv", false);
+      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv");
       if (qkv < 0) return P.rc;
       {
         OpDesc& o = c->ops[qkv];
@@ -503,8 +515,7 @@ static int build_plan(dec_ctx* c) {
       a.hd = hd;
       a.gs = hq / hkv;
       {
-        const OpDesc& p = c->ops[qkv];
-        a.qkv = PSet{p.out, p.S, p.out_stride, 0};
+        a.qkv = out_of(c->ops[qkv]);
       }
       a.nch = nch_dense;
       a.ntasks = hkv * a.nch;
@@ -521,7 +532,7 @@ static int build_plan(dec_ctx* c) {
       a.m_out = attn_buf[0];
       a.l_out = attn_buf[1];
       a.o_out = attn_buf[2];
-      if (dalloc(c, &a.o_fin, (size_t)hq * hd * 4)) return DEC_ERR_OOM;
+      if (dalloc(c, &a.o_fin, (size_t)2 * hq * hd * 8)) return DEC_ERR_OOM;
       a.kcache = c->kc[l];
       a.vcache = c->vc[l];
       a.rope_cos = c->rope_cos;
@@ -533,7 +544,7 @@ static int build_plan(dec_ctx* c) {
       OpDesc& oo = c->ops[o_op];
       oo.pro = PRO_SUM;  // the attention op's last chunk task per kv head combined the chunks
       oo.n = hq * hd;
-      oo.src = PSet{c->ops[attn].o_fin, 1, hq * hd, 0};
+      oo.src = PSet{c->ops[attn].o_fin, hq * hd, 0};
       oo.dep[0] = attn;
     } else {
       const int H = f.n_heads, nope = f.qk_nope, rd = f.qk_rope, vh = f.v_head, kvl = f.kv_lora;
@@ -547,15 +558,14 @@ static int build_plan(dec_ctx* c) {
         o.h_out = h_in[l];
       }
       Mat* qb = P.new_mat(DEC_W_Q_B, l, H * (nope + rd), f.q_lora, 1, 0);
-      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b", false);  // absorb_q reads one head per task
+      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b");
       if (s2 < 0) return P.rc;
       {
         OpDesc& o = c->ops[s2];
-        const OpDesc& p = c->ops[s1];
         o.pro = PRO_NORM_SUM;
         o.n = f.q_lora;
         o.gain = gainp(c, DEC_W_Q_A_NORM, l);
-        o.src = PSet{p.out, p.S, p.out_stride, 0};
+        o.src = out_of(c->ops[s1]);
         o.dep[0] = s1;
       }
       Mat* uk = P.new_mat(DEC_W_KV_B * 16 + 1, l, H * kvl, nope, 1, 1);  // W_UK^T view of kv_b
@@ -570,10 +580,9 @@ static int build_plan(dec_ctx* c) {
       }
       {
         OpDesc& o = c->ops[s3];
-        const OpDesc& p = c->ops[s2];
         o.pro = PRO_SUM;
         o.n = nope;
-        o.src = PSet{p.out, p.S, p.out_stride, 0};
+        o.src = out_of(c->ops[s2]);
         o.gstride = nope + rd;
         o.rows_per_group = kvl;
         o.dep[0] = s2;
@@ -583,8 +592,7 @@ static int build_plan(dec_ctx* c) {
         o.rope_cos = c->rope_cos;
         o.rope_sin = c->rope_sin;
         // an extra last task appends the step's latent row (normalised c, RoPE'd k_pe) to the cache
-        const OpDesc& p1 = c->ops[s1];
-        o.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
+        o.ckv = out_of(c->ops[s1], f.q_lora);
         o.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
         o.kcache = c->kc[l];
         group_tasks(o);
@@ -592,7 +600,6 @@ static int build_plan(dec_ctx* c) {
       }
       OpDesc a = P.base_op(OP_MLA, l);
       {
-        const OpDesc& p1 = c->ops[s1];
         a.H = H;
         a.kvl = kvl;
         a.rdim = rd;
@@ -600,7 +607,7 @@ static int build_plan(dec_ctx* c) {
         a.nch = nch_mla;
         a.ntasks = nch_mla;
         a.qc = qc;
-        a.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
+        a.ckv = out_of(c->ops[s1], f.q_lora);
         a.dep[0] = s3;
         a.pdep = s3;  // the producer streams the absorbed query
         a.max_seq = f.max_seq;
@@ -622,7 +629,7 @@ static int build_plan(dec_ctx* c) {
       a.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
       const int attn = P.push(a, "mla_attn");
       Mat* uv = P.new_mat(DEC_W_KV_B * 16 + 2, l, H * vh, kvl, 1, 2);  // W_UV view of kv_b
-      int s5 = P.gemv({{uv, -1, -1}}, kvl, l, false, "uv");
+      int s5 = P.gemv({{uv, -1, -1}}, kvl, l, true, "uv");
       if (s5 < 0) return P.rc;
       {
         OpDesc& o = c->ops[s5];
@@ -643,16 +650,14 @@ static int build_plan(dec_ctx* c) {
       if (o_op < 0) return P.rc;
       {
         OpDesc& o = c->ops[o_op];
-        const OpDesc& p = c->ops[s5];
         o.pro = PRO_SUM;
         o.n = H * vh;
-        o.src = PSet{p.out, p.S, p.out_stride, 0};
+        o.src = out_of(c->ops[s5]);
         o.dep[0] = s5;
       }
     }
     // ---- FFN
-    const OpDesc& oo = c->ops[o_op];
-    const PSet o_out{oo.out, oo.S, oo.out_stride, 0};
+    const PSet o_out = out_of(c->ops[o_op]);
     auto ffn_resid = [&](OpDesc& o, bool write_h) {
       o.pro = PRO_RESID_NORM;
       o.n = d;
@@ -674,11 +679,10 @@ static int build_plan(dec_ctx* c) {
       if (dn < 0) return P.rc;
       {
         OpDesc& o = c->ops[dn];
-        const OpDesc& p = c->ops[gu];
         o.pro = PRO_SWIGLU;
         o.n = ff;
-        o.gate = PSet{p.out, p.S, p.out_stride, 0};
-        o.up = PSet{p.out, p.S, p.out_stride, ff};
+        o.gate = out_of(c->ops[gu]);
+        o.up = out_of(c->ops[gu], ff);
         o.slot_stride = 0;
         o.dep[0] = gu;
       }
@@ -698,24 +702,31 @@ static int build_plan(dec_ctx* c) {
         CK(cudaMemsetAsync(o.rt_ids, 0, (size_t)k * 4, c->stream));
         CK(cudaMemsetAsync(o.rt_w, 0, (size_t)k * 4, c->stream));
       }
+      int* rids = c->ops[ro].rt_ids;
+      float* rw = c->ops[ro].rt_w;
+      // The shared expert's segments come first: its weights do not wait for the router, so
+      // the first tasks handed out stream while the router's top-k is decided.  Input group
+      // 0 is the shared expert's SwiGLU input, group j + 1 routed slot j's.
       Mat* eg = P.new_mat(DEC_W_EXP_GATE, l, eh, d, E, 0);
       Mat* eu = P.new_mat(DEC_W_EXP_UP, l, eh, d, E, 0);
-      Mat* sg = nullptr;
-      Mat* su = nullptr;
-      std::vector<SegSpec> segs;
+      Mat* ed = P.new_mat(DEC_W_EXP_DOWN, l, d, eh, E, 0);
+      std::vector<SegSpec> segs, dsegs;
+      const int g0 = f.n_shared > 0 ? 1 : 0;  // group of routed slot 0
+      if (f.n_shared > 0) {
+        Mat* sg = P.new_mat(DEC_W_SH_GATE, l, eh * f.n_shared, d, 1, 0);
+        Mat* su = P.new_mat(DEC_W_SH_UP, l, eh * f.n_shared, d, 1, 0);
+        Mat* sd = P.new_mat(DEC_W_SH_DOWN, l, d, eh * f.n_shared, 1, 0);
+        segs.push_back({sg, -1, 0});
+        segs.push_back({su, -1, 0});
+        dsegs.push_back({sd, -1, 0});
+      }
       for (int j = 0; j < k; ++j) {
         segs.push_back({eg, j, 0});
         segs.push_back({eu, j, 0});
-      }
-      if (f.n_shared > 0) {
-        sg = P.new_mat(DEC_W_SH_GATE, l, eh * f.n_shared, d, 1, 0);
-        su = P.new_mat(DEC_W_SH_UP, l, eh * f.n_shared, d, 1, 0);
-        segs.push_back({sg, -1, 0});
-        segs.push_back({su, -1, 0});
+        dsegs.push_back({ed, j, g0 + j});
       }
       int egu = P.gemv(segs, d, l, false, "exp_gate|up");
       if (egu < 0) return P.rc;
-      int* rids = c->ops[ro].rt_ids;
       {
         OpDesc& o = c->ops[egu];
         ffn_resid(o, false);
@@ -724,38 +735,30 @@ static int build_plan(dec_ctx* c) {
         o.n_experts = E;
         o.top_k = k;
       }
-      Mat* ed = P.new_mat(DEC_W_EXP_DOWN, l, d, eh, E, 0);
-      Mat* sd = nullptr;
-      std::vector<SegSpec> dsegs;
-      for (int j = 0; j < k; ++j) dsegs.push_back({ed, j, j});
-      if (f.n_shared > 0) {
-        sd = P.new_mat(DEC_W_SH_DOWN, l, d, eh * f.n_shared, 1, 0);
-        dsegs.push_back({sd, -1, k});
-      }
-      int edn = P.gemv(dsegs, eh, l, false, "exp_down");
+      int edn = P.gemv(dsegs, eh, l, false, "exp_down", true);
       if (edn < 0) return P.rc;
       {
         OpDesc& o = c->ops[edn];
-        const OpDesc& p = c->ops[egu];
         o.pro = PRO_SWIGLU;
         o.n = eh;
-        o.gate = PSet{p.out, p.S, p.out_stride, 0};
-        o.up = PSet{p.out, p.S, p.out_stride, eh};
+        o.gate = out_of(c->ops[egu]);
+        o.up = out_of(c->ops[egu], eh);
         o.slot_stride = 2 * eh;
         o.dep[0] = egu;
+        o.dep[1] = ro;  // the slot weights it applies
         o.pdep = ro;
         o.rt_ids = rids;
+        o.rt_w = rw;
         o.n_experts = E;
         o.top_k = k;
       }
       lo[l].ffn_op = edn;
-      lo[l].router_op = ro;
       ++c->n_moe;
     }
   }
   // ---- LM head + argmax
   Mat* lm = P.new_mat(DEC_W_LM_HEAD, -1, V, d, 1, 0);
-  int lmop = P.gemv({{lm, -1, 0}}, d, -1, true, "lm_head");
+  int lmop = P.gemv({{lm, -1, 0}}, d, -1, true, "lm_head", false, true);
   if (lmop < 0) return P.rc;
   {
     OpDesc& o = c->ops[lmop];
@@ -781,34 +784,21 @@ static int build_plan(dec_ctx* c) {
   return DEC_OK;
 }
 
-// ---------------------------------------------------------- task lists
-// Each op's tasks are cut into n_ctas contiguous runs, one per CTA, starting
-// at a CTA that rotates from op to op so that the remainders spread evenly.
-// Contiguous runs keep a CTA on one input group (expert slot, head) so that
-// the prologue building that group's input runs once per CTA, not per task.
-static int assign_tasks(dec_ctx* c) {
-  std::vector<std::vector<int2>> lists(c->n_ctas);
-  const int nc = c->n_ctas;
-  int rr = 0;
-  for (int op = 0; op < (int)c->ops.size(); ++op) {
-    const long long n = c->ops[op].ntasks;
-    for (int i = 0; i < nc; ++i) {
-      const int b = (rr + i) % nc;
-      for (long long t = i * n / nc; t < (i + 1) * n / nc; ++t) lists[b].push_back(make_int2(op, (int)t));
-    }
-    rr = (int)((rr + n) % nc);
+// ---------------------------------------------------------- task cursors
+// Every op gets one cursor per task group (two copies, for alternate steps), and its
+// first record in the trace buffer.
+static int setup_cursors(dec_ctx* c) {
+  int ncur = 0, trace = 0;
+  for (auto& o : c->ops) {
+    if (o.ngroups < 1) o.ngroups = 1;
+    o.cur_off = ncur;
+    o.trace_base = trace;
+    ncur += o.ngroups;
+    trace += o.ntasks;
   }
-  std::vector<int2> flat;
-  c->task_off.assign(c->n_ctas + 1, 0);
-  for (int b = 0; b < c->n_ctas; ++b) {
-    c->task_off[b] = (int)flat.size();
-    flat.insert(flat.end(), lists[b].begin(), lists[b].end());
-  }
-  c->task_off[c->n_ctas] = (int)flat.size();
-  if (dalloc(c, &c->d_tasks, flat.size() * sizeof(int2))) return DEC_ERR_OOM;
-  if (dalloc(c, &c->d_task_off, c->task_off.size() * sizeof(int))) return DEC_ERR_OOM;
-  CK(cudaMemcpy(c->d_tasks, flat.data(), flat.size() * sizeof(int2), cudaMemcpyHostToDevice));
-  CK(cudaMemcpy(c->d_task_off, c->task_off.data(), c->task_off.size() * sizeof(int), cudaMemcpyHostToDevice));
+  c->n_cursors = ncur;
+  if (dalloc(c, &c->d_cursors, (size_t)2 * ncur * 4)) return DEC_ERR_OOM;
+  c->accs.push_back({c->d_cursors, (size_t)2 * ncur * 4});  // cleared with the accumulators
   return DEC_OK;
 }
 
@@ -872,7 +862,7 @@ static int validate(const dec_config* f, dec_ctx* c) {
 static int check_work_area(dec_ctx* c) {
   // The prologues read partial sums with 16-byte loads: every vector they read
   // must start, and every split must be strided, at a multiple of 4 floats.
-  auto al = [](const PSet& p) { return !p.ptr || (p.off % 4 == 0 && p.stride % 4 == 0); };
+  auto al = [](const PSet& p) { return !p.acc || (p.off % 4 == 0 && p.stride % 4 == 0); };
   for (size_t i = 0; i < c->ops.size(); ++i) {
     const OpDesc& o = c->ops[i];
     const char* nm = c->op_names[i].c_str();
@@ -880,8 +870,8 @@ static int check_work_area(dec_ctx* c) {
     const int cap = o.pro == PRO_MLA_COMBINE ? kCombineOff : kWorkBytes;
     if ((long long)o.Kpad * (o.in_bf16 ? 2 : 4) > cap)
       return fail(c, DEC_ERR_UNSUPPORTED, "input vector of op %zu (%s) exceeds the work area", i, nm);
-    if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.add2) || !al(o.routed) || !al(o.src) || !al(o.gate) ||
-        !al(o.up) || o.routed_slot_stride % 4 || o.slot_stride % 4 || o.gstride % 4 || o.hdim % 4)
+    if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.src) || !al(o.gate) || !al(o.up) || o.slot_stride % 4 ||
+        o.gstride % 4 || o.hdim % 4)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): vector lengths and offsets must be multiples of 4", i, nm);
     if (o.pro == PRO_MLA_COMBINE && o.nch > kMaxCombine)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): too many split-KV chunks", i, nm);
@@ -892,6 +882,10 @@ static int check_work_area(dec_ctx* c) {
 static void free_all(dec_ctx* c) {
   if (c->graph) cudaGraphExecDestroy(c->graph);
   c->graph = nullptr;
+  if (c->gen_done) cudaEventDestroy(c->gen_done);
+  c->gen_done = nullptr;
+  if (c->h_map) cudaFreeHost(c->h_map);
+  c->h_map = nullptr;
   for (void* p : c->allocs) cudaFree(p);
   c->allocs.clear();
   if (c->staging) cudaFree(c->staging);
@@ -999,16 +993,30 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
       }
     }
   }
+  if ((rc = setup_cursors(c))) return rc;
   if ((rc = upload_ops(c))) return rc;
-  if ((rc = assign_tasks(c))) return rc;
   if ((rc = dalloc(c, &c->d_state, sizeof(StepState)))) return rc;
+  if ((rc = dalloc(c, &c->d_gen, sizeof(GenState)))) return rc;
+  CK(cudaMemsetAsync(c->d_gen, 0, sizeof(GenState), c->stream));
+  {  // the token ring the device writes and the host reads while a generation runs
+    const size_t mb = 16 + (size_t)f.max_seq * 4;
+    cudaError_t e = cudaHostAlloc(&c->h_map, mb, cudaHostAllocMapped);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      c->h_map = nullptr;
+      return fail(c, DEC_ERR_OOM, "mapped host memory for the token ring: %s", cudaGetErrorString(e));
+    }
+    memset(c->h_map, 0, mb);
+    CK(cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->d_map), c->h_map, 0));
+    CK(cudaEventCreateWithFlags(&c->gen_done, cudaEventDisableTiming));
+  }
   if ((rc = dalloc(c, &c->d_started, 4))) return rc;
   if ((rc = dalloc(c, &c->d_status, sizeof(Status)))) return rc;
   if (f.flags & DEC_FLAG_TRACE) {
     int total = 0;
     for (auto& o : c->ops) total += o.ntasks;
     c->trace_cap = total;
-    if ((rc = dalloc(c, &c->d_trace, (2 + 7 * (size_t)total) * 8))) return rc;
+    if ((rc = dalloc(c, &c->d_trace, (2 + 9 * (size_t)total) * 8))) return rc;
   }
   // bytes a step reads from the weight store (active weights + scales)
   for (auto& kv : c->mats) {
@@ -1038,6 +1046,7 @@ extern "C" const char* dec_last_error(const dec_ctx* c) { return c ? c->err.c_st
 
 extern "C" int dec_set_stream(dec_ctx* c, void* stream) {
   if (!c) return DEC_ERR_INVALID_ARG;
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is running; call dec_generate_wait");
   CK(cudaStreamSynchronize(c->stream));
   if (c->graph) {
     cudaGraphExecDestroy(c->graph);
@@ -1059,11 +1068,14 @@ extern "C" int dec_reset(dec_ctx* c) {
   cudaStreamSynchronize(c->stream);
   (void)cudaGetLastError();
   CK(cudaMemsetAsync(c->d_counters, 0, c->n_counters * 4, c->stream));
+  for (auto& a : c->accs) CK(cudaMemsetAsync(a.first, 0, a.second, c->stream));
   CK(cudaMemsetAsync(c->d_started, 0, 4, c->stream));
   CK(cudaMemsetAsync(c->d_status, 0, sizeof(Status), c->stream));
+  CK(cudaMemsetAsync(c->d_gen, 0, sizeof(GenState), c->stream));
   StepState st{1, 0, 0, 0};
   CK(cudaMemcpyAsync(c->d_state, &st, sizeof st, cudaMemcpyHostToDevice, c->stream));
   CK(cudaStreamSynchronize(c->stream));
+  c->generating = false;
   c->pos = 0;
   c->epoch = 1;
   c->have_ctx = false;
@@ -1119,7 +1131,7 @@ static int load_matrix(dec_ctx* c, Mat& m, int expert, const void* data, const f
   uint8_t* dst = m.w + (size_t)expert * m.tile_bytes;
   const long long total16 = (long long)(m.tile_bytes / 16);
   const int grid = (int)std::min<long long>((total16 + 255) / 256, 148 * 16);
-  relayout16<<<std::max(grid, 1), 256, 0, c->stream>>>(src, m.N, m.K, m.wb, m.R, m.S, m.nst, m.kcb, total16, dst);
+  relayout16<<<std::max(grid, 1), 256, 0, c->stream>>>(src, m.N, m.K, m.wb, m.R, m.nst, m.kcb, total16, dst);
   CK(cudaGetLastError());
   if (m.sc_count) CK(cudaMemcpyAsync(m.sc + (size_t)expert * m.sc_count, scales, m.sc_count * 4, cudaMemcpyDefault, c->stream));
   CK(cudaStreamSynchronize(c->stream));
@@ -1142,7 +1154,7 @@ static int load_kvb(dec_ctx* c, int layer, const void* data, const float* scales
     Mat& m = c->mats[{DEC_W_KV_B * 16 + mode, layer}];
     const long long total = (long long)m.tile_bytes;
     const int grid = (int)std::min<long long>((total + 255) / 256, 148 * 16);
-    relayout_kvb<<<std::max(grid, 1), 256, 0, c->stream>>>(src, mode, m.N, m.K, m.wb, m.R, m.S, m.nst, m.kcb, total,
+    relayout_kvb<<<std::max(grid, 1), 256, 0, c->stream>>>(src, mode, m.N, m.K, m.wb, m.R, m.nst, m.kcb, total,
                                                            nope, vh, kvl, m.w);
     CK(cudaGetLastError());
   }
@@ -1174,6 +1186,7 @@ static int load_kvb(dec_ctx* c, int layer, const void* data, const float* scales
 
 extern "C" int dec_load_weights(dec_ctx* c, const dec_tensor* t, int n) {
   if (!c || (!t && n > 0) || n < 0) return DEC_ERR_INVALID_ARG;
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is running; call dec_generate_wait");
   CK(cudaSetDevice(c->cfg.device));
   // Device sources may have been produced on any stream: read them only after
   // all work already submitted to the device has finished.
@@ -1238,6 +1251,7 @@ static bool all_loaded(dec_ctx* c) {
 // ------------------------------------------------------------------ cache
 extern "C" int dec_set_kv_cache(dec_ctx* c, const void* k_or_latent, const void* v_or_pe, int32_t n_tokens) {
   if (!c) return DEC_ERR_INVALID_ARG;
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is running; call dec_generate_wait");
   const dec_config& f = c->cfg;
   if (n_tokens < 0) return fail(c, DEC_ERR_INVALID_ARG, "n_tokens < 0");
   if (n_tokens >= f.max_seq) return fail(c, DEC_ERR_CAPACITY, "context of %d tokens needs max_seq > %d", n_tokens, n_tokens);
@@ -1299,8 +1313,8 @@ static KParams kparams(dec_ctx* c, int persistent, int op, int tok_in) {
   memset(&P, 0, sizeof P);
   P.ops = c->d_ops;
   P.nops = (int)c->ops.size();
-  P.tasks = c->d_tasks;
-  P.task_off = c->d_task_off;
+  P.cursors = c->d_cursors;
+  P.ncur = c->n_cursors;
   P.counters = c->d_counters;
   P.state = c->d_state;
   P.started = c->d_started;
@@ -1314,6 +1328,11 @@ static KParams kparams(dec_ctx* c, int persistent, int op, int tok_in) {
   P.trace_cap = c->trace_cap;
   P.tok_in = tok_in;
   P.test_stall = (c->cfg.flags & DEC_FLAG_TEST_STALL) ? 1 : 0;
+  P.n_steps = 1;
+  P.gen = c->d_gen;
+  P.tok_count = reinterpret_cast<unsigned*>(c->d_map);
+  P.stop_word = reinterpret_cast<const int*>(c->d_map + 4);
+  P.tok_ring = reinterpret_cast<int*>(c->d_map + 16);
   return P;
 }
 
@@ -1346,7 +1365,8 @@ static int ensure_graph(dec_ctx* c) {
 
 static int enqueue_step(dec_ctx* c, int32_t token_id) {
   const dec_config& f = c->cfg;
-  if (c->poisoned) return fail(c, DEC_ERR_STATE, "context poisoned by an earlier device timeout; call dec_reset");
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is running; call dec_generate_wait");
+  if (c->poisoned) return fail(c, DEC_ERR_STATE, "context poisoned by an earlier device failure; call dec_reset");
   if (!all_loaded(c)) return fail(c, DEC_ERR_STATE, "not every weight tensor has been loaded");
   if (!c->have_ctx) return fail(c, DEC_ERR_STATE, "no context: call dec_set_kv_cache first");
   if (c->pos + 1 > f.max_seq) return fail(c, DEC_ERR_CAPACITY, "position %d reaches max_seq %d", c->pos, f.max_seq);
@@ -1354,7 +1374,7 @@ static int enqueue_step(dec_ctx* c, int32_t token_id) {
   if (token_id < 0 && c->epoch == 1)  // epoch 1: no step since the last reset / context install
     return fail(c, DEC_ERR_STATE, "no previous greedy token to feed back");
   CK(cudaSetDevice(f.device));
-  if (c->d_trace) CK(cudaMemsetAsync(c->d_trace, 0, (2 + 7 * (size_t)c->trace_cap) * 8, c->stream));
+  if (c->d_trace) CK(cudaMemsetAsync(c->d_trace, 0, (2 + 9 * (size_t)c->trace_cap) * 8, c->stream));
   int rc = DEC_OK;
   if (c->mode == DEC_PERSISTENT) {
     KParams P = kparams(c, 1, -1, token_id);
@@ -1386,8 +1406,11 @@ static int finish(dec_ctx* c, float* out_logits, int32_t* out_next) {
   c->pending = 0;
   if (st.code != 0) {
     c->poisoned = true;
-    return fail(c, DEC_ERR_TIMEOUT, "device wait timed out (cta %d, op %d '%s', task %d)", st.cta, st.op,
-                st.op >= 0 && st.op < (int)c->op_names.size() ? c->op_names[st.op].c_str() : "?", st.task);
+    const char* nm = st.op >= 0 && st.op < (int)c->op_names.size() ? c->op_names[st.op].c_str() : "?";
+    if (st.code == 2)
+      return fail(c, DEC_ERR_NUMERIC, "non-finite logit (cta %d, op %d '%s', task %d)", st.cta, st.op, nm, st.task);
+    return fail(c, DEC_ERR_TIMEOUT, "device wait timed out (cta %d, op %d '%s', task %d)", st.cta, st.op, nm,
+                st.task);
   }
   if (out_next) *out_next = ss.last;
   if (out_logits) {
@@ -1414,8 +1437,123 @@ extern "C" int dec_sync(dec_ctx* c, float* out_logits, int32_t* out_next_token) 
   return finish(c, out_logits, out_next_token);
 }
 
+// ------------------------------------------------------------- generation
+// A decode lifetime with the host out of the loop: in DEC_PERSISTENT mode one kernel
+// launch runs every step, feeding each greedy token back on the device and writing it
+// to a host-mapped ring as soon as it is known (InferenceX article, "what TileRT is":
+// the host launches once for the whole decode).  The other modes run the same steps
+// one launch per step (per op, or a CUDA graph per step) with a host check of the stop
+// condition after each step: the ablation of what the single launch removes.
+extern "C" int dec_generate_async(dec_ctx* c, int32_t token_id, int32_t n_steps, int32_t stop_token) {
+  if (!c) return DEC_ERR_INVALID_ARG;
+  const dec_config& f = c->cfg;
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is already running");
+  if (n_steps < 1) return fail(c, DEC_ERR_INVALID_ARG, "n_steps < 1");
+  if (c->pos + n_steps > f.max_seq)
+    return fail(c, DEC_ERR_CAPACITY, "position %d + %d steps exceeds max_seq %d", c->pos, n_steps, f.max_seq);
+  if (c->poisoned) return fail(c, DEC_ERR_STATE, "context poisoned by an earlier device failure; call dec_reset");
+  if (!all_loaded(c)) return fail(c, DEC_ERR_STATE, "not every weight tensor has been loaded");
+  if (!c->have_ctx) return fail(c, DEC_ERR_STATE, "no context: call dec_set_kv_cache first");
+  if (token_id >= f.vocab) return fail(c, DEC_ERR_INVALID_ARG, "token %d >= vocab %d", token_id, f.vocab);
+  if (token_id < 0 && c->epoch == 1) return fail(c, DEC_ERR_STATE, "no previous greedy token to feed back");
+  CK(cudaSetDevice(f.device));
+  CK(cudaStreamSynchronize(c->stream));  // the ring and stop word are reused: nothing may still write them
+  *h_count(c) = 0;
+  *h_stop(c) = 0;
+  GenState g{1, c->epoch, stop_token, 0};
+  CK(cudaMemcpyAsync(c->d_gen, &g, sizeof g, cudaMemcpyHostToDevice, c->stream));
+  c->gen_epoch0 = c->epoch;
+  c->gen_steps = n_steps;
+  c->gen_stop_token = stop_token;
+  if (c->d_trace) CK(cudaMemsetAsync(c->d_trace, 0, (2 + 9 * (size_t)c->trace_cap) * 8, c->stream));
+  if (c->mode == DEC_PERSISTENT) {
+    KParams P = kparams(c, 1, -1, token_id);
+    P.n_steps = n_steps;
+    void* args[] = {&P};
+    CK(cudaLaunchCooperativeKernel(c->kernel, dim3(c->n_ctas), dim3(kThreads), args, kSmemBytes, c->stream));
+  } else {  // one launch per step; the host checks the stop condition after each
+    for (int i = 0; i < n_steps; ++i) {
+      int rc = c->mode == DEC_PER_OP ? launch_per_op(c, i == 0 ? token_id : -1) : DEC_OK;
+      if (c->mode == DEC_PER_OP_GRAPH) {
+        if ((rc = ensure_graph(c))) return rc;
+        if (i == 0 && token_id >= 0) {
+          set_int<<<1, 1, 0, c->stream>>>(&c->d_state->tok, token_id);
+          CK(cudaGetLastError());
+        }
+        CK(cudaGraphLaunch(c->graph, c->stream));
+      }
+      if (rc) return rc;
+      CK(cudaStreamSynchronize(c->stream));
+      const unsigned n = *h_count(c);
+      if (n < (unsigned)(i + 1) || (n > 0 && h_ring(c)[n - 1] == stop_token) || *h_stop(c)) break;
+    }
+  }
+  CK(cudaEventRecord(c->gen_done, c->stream));
+  c->generating = true;
+  return DEC_OK;
+}
+
+extern "C" int dec_generate_poll(dec_ctx* c, int32_t* out_tokens, int32_t cap, int32_t* out_count,
+                                 int32_t* out_done) {
+  if (!c || cap < 0 || (cap > 0 && !out_tokens)) return DEC_ERR_INVALID_ARG;
+  if (!c->generating) return fail(c, DEC_ERR_STATE, "no generation is running");
+  const unsigned n = *h_count(c);  // the device writes a ring entry before the count
+  for (unsigned i = 0; i < n && (int)i < cap; ++i) out_tokens[i] = h_ring(c)[i];
+  if (out_count) *out_count = (int32_t)n;
+  if (out_done) {
+    const cudaError_t e = cudaEventQuery(c->gen_done);
+    if (e != cudaSuccess && e != cudaErrorNotReady) return fail(c, DEC_ERR_CUDA, "%s", cudaGetErrorString(e));
+    (void)cudaGetLastError();
+    *out_done = e == cudaSuccess;
+  }
+  return DEC_OK;
+}
+
+extern "C" int dec_generate_stop(dec_ctx* c) {
+  if (!c) return DEC_ERR_INVALID_ARG;
+  *h_stop(c) = 1;
+  return DEC_OK;
+}
+
+extern "C" int dec_generate_wait(dec_ctx* c, int32_t* out_tokens, int32_t cap, int32_t* out_count) {
+  if (!c || cap < 0 || (cap > 0 && !out_tokens)) return DEC_ERR_INVALID_ARG;
+  if (!c->generating) return fail(c, DEC_ERR_STATE, "no generation is running");
+  CK(cudaSetDevice(c->cfg.device));
+  Status st;
+  StepState ss;
+  const GenState off{0, 0, -1, 0};
+  CK(cudaMemcpyAsync(&st, c->d_status, sizeof st, cudaMemcpyDeviceToHost, c->stream));
+  CK(cudaMemcpyAsync(&ss, c->d_state, sizeof ss, cudaMemcpyDeviceToHost, c->stream));
+  CK(cudaMemcpyAsync(c->d_gen, &off, sizeof off, cudaMemcpyHostToDevice, c->stream));
+  CK(cudaStreamSynchronize(c->stream));
+  c->generating = false;
+  const int done = ss.epoch - c->gen_epoch0;  // steps completed
+  c->pos += done;
+  c->epoch += done;
+  const unsigned n = *h_count(c);
+  for (unsigned i = 0; i < n && (int)i < cap; ++i) out_tokens[i] = h_ring(c)[i];
+  if (out_count) *out_count = (int32_t)n;
+  if (st.code != 0) {
+    c->poisoned = true;
+    const char* nm = st.op >= 0 && st.op < (int)c->op_names.size() ? c->op_names[st.op].c_str() : "?";
+    if (st.code == 2)
+      return fail(c, DEC_ERR_NUMERIC, "non-finite logit (cta %d, op %d '%s', task %d)", st.cta, st.op, nm, st.task);
+    return fail(c, DEC_ERR_TIMEOUT, "device wait timed out (cta %d, op %d '%s', task %d)", st.cta, st.op, nm,
+                st.task);
+  }
+  return DEC_OK;
+}
+
+extern "C" int dec_generate(dec_ctx* c, int32_t token_id, int32_t n_steps, int32_t stop_token, int32_t* out_tokens,
+                            int32_t* out_count) {
+  int rc = dec_generate_async(c, token_id, n_steps, stop_token);
+  if (rc) return rc;
+  return dec_generate_wait(c, out_tokens, n_steps, out_count);
+}
+
 extern "C" int dec_set_exec_mode(dec_ctx* c, int32_t mode) {
   if (!c || mode < DEC_PERSISTENT || mode > DEC_PER_OP_GRAPH) return DEC_ERR_INVALID_ARG;
+  if (c->generating) return fail(c, DEC_ERR_STATE, "a generation is running; call dec_generate_wait");
   CK(cudaStreamSynchronize(c->stream));
   c->mode = mode;
   if (mode == DEC_PER_OP_GRAPH) return ensure_graph(c);
@@ -1439,7 +1577,13 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
     uint8_t* o = reinterpret_cast<uint8_t*>(dst);
-    uint8_t* rows = nullptr;
+    uint8_t* rows = nullptr;  // MLA only: one layer's [n][kv_lora | qk_rope] rows
+    struct FreeRows {         // freed on every return, the CK(...) error returns included
+      uint8_t*& p;
+      ~FreeRows() {
+        if (p) cudaFree(p);
+      }
+    } free_rows{rows};
     for (int l = 0; l < f.n_layers && n > 0; ++l) {
       if (!mla) {
         const size_t row = (size_t)n * f.head_dim * c->eb, sp = (size_t)f.max_seq * f.head_dim * c->eb;
@@ -1463,7 +1607,11 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
         CK(cudaMemcpy2D(o + nl * lat + (size_t)l * n * pe, pe, rows + lat, rowb, pe, n, cudaMemcpyDeviceToHost));
       }
     }
-    if (rows) CK(cudaFree(rows));
+    if (rows) {
+      const cudaError_t e = cudaFree(rows);
+      rows = nullptr;
+      if (e != cudaSuccess) return fail(c, DEC_ERR_CUDA, "dump scratch: %s", cudaGetErrorString(e));
+    }
     return DEC_OK;
   }
   if (what == DEC_DUMP_ROUTES) {
@@ -1479,7 +1627,7 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     unsigned long long hdr[2];
     CK(cudaMemcpy(hdr, c->d_trace, 16, cudaMemcpyDeviceToHost));
     const size_t nrec = std::min<size_t>((unsigned)hdr[0], (size_t)c->trace_cap);
-    const size_t need = nrec * 40;
+    const size_t need = nrec * 48;
     if (out_bytes) *out_bytes = need;
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
@@ -1488,11 +1636,11 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
   }
   if (what == DEC_DUMP_TRACE_PRODUCER) {
     if (!c->d_trace) return fail(c, DEC_ERR_STATE, "context created without DEC_FLAG_TRACE");
-    const size_t need = (size_t)c->trace_cap * 16;
+    const size_t need = (size_t)c->trace_cap * 24;
     if (out_bytes) *out_bytes = need;
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
-    CK(cudaMemcpy(dst, c->d_trace + 2 + 5 * (size_t)c->trace_cap, need, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(dst, c->d_trace + 2 + 6 * (size_t)c->trace_cap, need, cudaMemcpyDeviceToHost));
     return DEC_OK;
   }
   if (what == DEC_DUMP_PLAN) {
@@ -1501,8 +1649,9 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     for (size_t i = 0; i < c->ops.size(); ++i) {
       const OpDesc& o = c->ops[i];
       snprintf(line, sizeof line,
-               "%zu %s layer=%d kind=%d tasks=%d K=%d Kpad=%d kcb=%d R=%d S=%d nst=%d segs=%d dep=%d,%d pdep=%d nch=%d\n",
-               i, c->op_names[i].c_str(), o.layer, o.kind, o.ntasks, o.K, o.Kpad, o.kcb, o.R, o.S, o.nst, o.nsegs,
+               "%zu %s layer=%d kind=%d tasks=%d K=%d Kpad=%d kcb=%d R=%d acc=%d nst=%d segs=%d dep=%d,%d pdep=%d nch=%d\n",
+               i, c->op_names[i].c_str(), o.layer, o.kind, o.ntasks, o.K, o.Kpad, o.kcb, o.R, o.acc ? 1 : 0, o.nst_total,
+               o.nsegs,
                o.dep[0], o.dep[1], o.pdep, o.nch);
       s += line;
     }
@@ -1515,6 +1664,17 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     memcpy(dst, s.c_str(), s.size() + 1);
     return DEC_OK;
   }
+  if (what == DEC_DUMP_STATUS) {
+    const size_t need = sizeof(Status) + sizeof(StepState);
+    static_assert(sizeof(Status) + sizeof(StepState) == 48, "status dump layout");
+    if (out_bytes) *out_bytes = need;
+    if (!dst) return DEC_OK;
+    if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
+    CK(cudaMemcpy(dst, c->d_status, sizeof(Status), cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(reinterpret_cast<uint8_t*>(dst) + sizeof(Status), c->d_state, sizeof(StepState),
+                  cudaMemcpyDeviceToHost));
+    return DEC_OK;
+  }
   if (what == DEC_DUMP_WEIGHTS) {
     if (out_bytes) *out_bytes = 16;
     if (!dst) return DEC_OK;
@@ -1525,9 +1685,21 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
   }
   if (what >= DEC_DUMP_OP && what < DEC_DUMP_OP + (int)c->ops.size()) {
     const OpDesc& o = c->ops[what - DEC_DUMP_OP];
+    if (o.kind == OP_GEMV && o.acc) {  // the last step's accumulator copy, converted to fp32
+      const size_t need = (size_t)o.out_stride * 4;
+      if (out_bytes) *out_bytes = need;
+      if (!dst) return DEC_OK;
+      if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
+      std::vector<long long> a(o.out_stride);
+      const int par = (c->epoch - 1) & 1;
+      CK(cudaMemcpy(a.data(), o.acc + (size_t)par * o.out_stride, a.size() * 8, cudaMemcpyDeviceToHost));
+      float* f32 = reinterpret_cast<float*>(dst);
+      for (size_t i = 0; i < a.size(); ++i) f32[i] = (float)((double)a[i] * (1.0 / 1099511627776.0));
+      return DEC_OK;
+    }
     std::vector<std::pair<const float*, size_t>> parts;
     if (o.kind == OP_GEMV) {
-      parts.push_back({o.out, (size_t)o.S * o.out_stride});
+      parts.push_back({o.out, (size_t)o.out_stride});
     } else if (o.kind == OP_ATTN || o.kind == OP_MLA) {
       const int heads = o.kind == OP_ATTN ? o.hq : o.H, dim = o.kind == OP_ATTN ? o.hd : o.kvl;
       parts.push_back({o.m_out, (size_t)heads * o.nch});

@@ -170,16 +170,22 @@ extern "C" int dec_attention_noalloc(const float* q, const void* k_cache, const 
                                      int32_t n_kv_heads, int32_t head_dim, int32_t n_pos, int32_t cache_stride,
                                      float* out, void* stream) {
   if (!q || !k_cache || !v_cache || !out) return DEC_ERR_INVALID_ARG;
+  // K and V rows are read with 16-byte loads; q and out with 4-byte ones
+  if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15) return DEC_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 3) return DEC_ERR_INVALID_ARG;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || n_heads / n_kv_heads > 8) return DEC_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return DEC_ERR_INVALID_ARG;
   if (n_pos < 1 || cache_stride < n_pos) return DEC_ERR_INVALID_ARG;
-  // about one block per SM of a B200, at most 64 chunks (one warp combines them)
+  // About one block per SM of a B200, at most 64 chunks (one warp combines them).  With
+  // n_kv_heads <= 148 this keeps n_heads * nch <= 8 * 148 rows of partials, far inside the
+  // scratch; only very many kv heads (nch = 1) can exceed it.
   int nch = 148 / n_kv_heads;
   if (nch < 1) nch = 1;
   if (nch > 64) nch = 64;
   if (nch > n_pos) nch = n_pos;
-  while (nch > 1 && (long long)n_heads * nch * (head_dim + 2) > kScratchFloats) --nch;
   if ((long long)n_heads * nch * (head_dim + 2) > kScratchFloats) return DEC_ERR_CAPACITY;
+  // A launch error of this call must not be confused with one the caller left pending.
+  if (cudaPeekAtLastError() != cudaSuccess) return DEC_ERR_CUDA;
   float* scratch = nullptr;
   int rc = scratch_address(&scratch);
   if (rc) return rc;

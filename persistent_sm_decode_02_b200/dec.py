@@ -22,6 +22,7 @@ DEC_ERR_OOM = -4
 DEC_ERR_CUDA = -5
 DEC_ERR_TIMEOUT = -6
 DEC_ERR_UNSUPPORTED = -7
+DEC_ERR_NUMERIC = -8
 
 DEC_ARCH_DENSE = 0
 DEC_ARCH_MLA_MOE = 1
@@ -44,11 +45,13 @@ DEC_DUMP_TRACE = 3
 DEC_DUMP_PLAN = 4
 DEC_DUMP_WEIGHTS = 5
 DEC_DUMP_TRACE_PRODUCER = 6
+DEC_DUMP_STATUS = 7
 DEC_DUMP_OP = 100
 
 EXPORTED = ["dec_create", "dec_load_weights", "dec_set_kv_cache", "dec_step", "dec_step_async", "dec_sync",
             "dec_reset", "dec_destroy", "dec_set_stream", "dec_set_exec_mode", "dec_position", "dec_debug_dump",
-            "dec_last_error", "dec_attention_noalloc"]
+            "dec_last_error", "dec_attention_noalloc", "dec_generate_async", "dec_generate_poll",
+            "dec_generate_stop", "dec_generate_wait", "dec_generate"]
 
 
 class dec_config(ctypes.Structure):
@@ -92,6 +95,11 @@ def load_library():
             "dec_debug_dump": [P, ctypes.c_int32, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)],
             "dec_attention_noalloc": [P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                       ctypes.c_int32, P, P],
+            "dec_generate_async": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32],
+            "dec_generate_poll": [P, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32)],
+            "dec_generate_stop": [P],
+            "dec_generate_wait": [P, P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)],
+            "dec_generate": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, ctypes.POINTER(ctypes.c_int32)],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -177,6 +185,26 @@ def dec_attention_noalloc(q, k_cache, v_cache, n_heads, n_kv_heads, head_dim, n_
                                                 cache_stride, out, stream)
 
 
+def dec_generate_async(ctx, token_id, n_steps, stop_token):
+    return load_library().dec_generate_async(ctx, token_id, n_steps, stop_token)
+
+
+def dec_generate_poll(ctx, out_tokens, cap, out_count, out_done):
+    return load_library().dec_generate_poll(ctx, out_tokens, cap, out_count, out_done)
+
+
+def dec_generate_stop(ctx):
+    return load_library().dec_generate_stop(ctx)
+
+
+def dec_generate_wait(ctx, out_tokens, cap, out_count):
+    return load_library().dec_generate_wait(ctx, out_tokens, cap, out_count)
+
+
+def dec_generate(ctx, token_id, n_steps, stop_token, out_tokens, out_count):
+    return load_library().dec_generate(ctx, token_id, n_steps, stop_token, out_tokens, out_count)
+
+
 # ---- convenience
 def config_from_workload(w: dict, exec_mode=DEC_PERSISTENT, device=0, timeout_us=0, flags=0, n_ctas=0):
     c = dec_config()
@@ -244,6 +272,32 @@ class Decoder:
 
     def reset(self):
         _chk(self.ctx, dec_reset(self.ctx))
+
+    def generate(self, token_id: int, n_steps: int, stop_token: int = -1):
+        """Tokens of a whole generation (one kernel launch in DEC_PERSISTENT mode)."""
+        out = (ctypes.c_int32 * max(1, n_steps))()
+        n = ctypes.c_int32(0)
+        _chk(self.ctx, dec_generate(self.ctx, token_id, n_steps, stop_token, out, ctypes.byref(n)))
+        return list(out[:n.value])
+
+    def generate_async(self, token_id: int, n_steps: int, stop_token: int = -1):
+        _chk(self.ctx, dec_generate_async(self.ctx, token_id, n_steps, stop_token))
+
+    def generate_poll(self, cap: int = 0):
+        """(tokens so far, done) of the running generation, without waiting."""
+        out = (ctypes.c_int32 * max(1, cap))()
+        n, done = ctypes.c_int32(0), ctypes.c_int32(0)
+        _chk(self.ctx, dec_generate_poll(self.ctx, out, cap, ctypes.byref(n), ctypes.byref(done)))
+        return list(out[:min(n.value, cap)]), bool(done.value)
+
+    def generate_stop(self):
+        _chk(self.ctx, dec_generate_stop(self.ctx))
+
+    def generate_wait(self, cap: int):
+        out = (ctypes.c_int32 * max(1, cap))()
+        n = ctypes.c_int32(0)
+        _chk(self.ctx, dec_generate_wait(self.ctx, out, cap, ctypes.byref(n)))
+        return list(out[:min(n.value, cap)])
 
     def set_exec_mode(self, mode):
         _chk(self.ctx, dec_set_exec_mode(self.ctx, mode))

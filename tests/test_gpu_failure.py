@@ -138,3 +138,57 @@ def test_a_stream_given_to_the_decoder_stays_the_callers(pkg):
         assert d2.step(3) == tok
     finally:
         d2.close()
+
+
+def test_nonfinite_lm_logits_are_reported(pkg):
+    """A NaN final-norm gain (a corrupt weight, injected on the host) makes every logit NaN: the
+    step returns DEC_ERR_NUMERIC instead of a greedy token, the context stays poisoned until
+    dec_reset, and with the weight restored the decoder works again."""
+    w = workloads.get("small_dense_bf16")
+    d = _decoder(pkg, w)
+    try:
+        k, v = sdev.synthetic_cache_device(w)
+        good, _ = sdev.gen_tensor(w, [s for s in workloads.weight_specs(w) if s["name"] == "final_norm"][0])
+        bad = np.full(w["d_model"], np.nan, np.float32)
+        d.load("final_norm", -1, bad.ctypes.data, bad.nbytes)
+        d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        with pytest.raises(pkg.DecError) as e:
+            d.step(3)
+        assert e.value.code == pkg.dec.DEC_ERR_NUMERIC
+        assert "final" in str(e.value)
+        with pytest.raises(pkg.DecError) as e:
+            d.step(3)
+        assert e.value.code == pkg.dec.DEC_ERR_STATE
+        d.load("final_norm", -1, good.data_ptr(), good.numel() * 4)
+        d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        assert 0 <= d.step(3) < w["vocab"]
+    finally:
+        d.close()
+
+
+def test_nonfinite_router_logits_are_reported(pkg):
+    """One router row of E4M3 NaN codes (0x7F) in the first MoE layer gives that expert a NaN
+    logit: the router's top-k reports it (DEC_ERR_NUMERIC, op 'router') instead of silently
+    routing around it."""
+    w = workloads.get("small_mla_moe_fp8")
+    d = _decoder(pkg, w)
+    try:
+        k, v = sdev.synthetic_cache_device(w)
+        layer = w["n_dense_layers"]
+        spec = [s for s in workloads.weight_specs(w) if s["name"] == "router" and s["layer"] == layer][0]
+        q, sc = sdev.gen_tensor(w, spec)
+        q = q.view(spec["shape"]).clone()
+        q[3] = 0x7F
+        d.load("router", layer, q.data_ptr(), q.numel(), sc.data_ptr())
+        d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        with pytest.raises(pkg.DecError) as e:
+            d.step(3)
+        assert e.value.code == pkg.dec.DEC_ERR_NUMERIC
+        assert "router" in str(e.value)
+        d.reset()
+        q0, sc0 = sdev.gen_tensor(w, spec)
+        d.load("router", layer, q0.data_ptr(), q0.numel(), sc0.data_ptr())
+        d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+        assert 0 <= d.step(3) < w["vocab"]
+    finally:
+        d.close()

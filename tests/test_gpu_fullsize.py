@@ -6,8 +6,8 @@ layers (first, middle, last) and the LM head is checked against the oracle op
 evaluated on the GPU's own inputs (rebuilt from the step's dumps), which holds
 at any size: all ops agree to ~1e-7 relative except where a bf16 rounding flips.
 The router's chosen experts must be the top-k of the GPU's router logits
-(exempt below a 1e-4 margin), and the dense bf16 workload also matches the
-oracle's greedy token end to end.
+(exempt below a 1e-4 margin).  End-to-end parity of the same workloads, teacher
+forced over several steps, is in test_gpu_fullsize_e2e.py.
 """
 import math
 
@@ -57,8 +57,8 @@ class Step:
         return np.frombuffer(self.d.dump(self.pkg.dec.DEC_DUMP_OP + i), np.float32).astype(np.float64)
 
     def out(self, layer, name):
-        i = self.by_layer[layer][name]
-        return self.raw(i).reshape(int(self.plan[i][1]["S"]), -1).sum(0)
+        """The op's output vector (row tiles split among CTAs are already summed on the device)."""
+        return self.raw(self.by_layer[layer][name])
 
     def combine(self, layer, name, heads, dim):
         i = self.by_layer[layer][name]
@@ -76,17 +76,11 @@ class Step:
 
 
 def _ffn_out(st, w, l, moe_l):
-    """GPU FFN output of layer l (dense down sum, or routed + shared experts with router weights)."""
+    """GPU FFN output of layer l: the dense down projection, or the MoE layer's accumulator (routed
+    experts weighted by the router, plus the shared expert), which the expert-down op dumps."""
     if w["arch"] == "dense" or l < w["n_dense_layers"]:
         return st.out(l, "down")
-    d = w["d_model"]
-    r = st.out(l, "router")
-    idx, wts = om.route_topk(r, w["top_k"])
-    dn = st.out(l, "exp_down")
-    f = sum(wts[j] * dn[j * d:(j + 1) * d] for j in range(w["top_k"]))
-    if w["n_shared"]:
-        f = f + dn[w["top_k"] * d:(w["top_k"] + 1) * d]
-    return f
+    return st.out(l, "exp_down")
 
 
 @pytest.mark.parametrize("name", ["dense_gqa_bf16_1k", "dense_gqa_fp8_8k", "moe_mla_fp8_1k", "moe_mla_fp8_8k"])
@@ -118,7 +112,7 @@ def test_fullsize_sampled_ops(name):
                     K = kv[: kv.size // 2].reshape(L, hkv, n, hd)[l]
                     V = kv[kv.size // 2:].reshape(L, hkv, n, hd)[l]
                     q = R(rope(qkv[: hq * hd].reshape(hq, hd), p, th))
-                    o = np.stack([softmax(K[i * hkv // hq] @ q[i] / math.sqrt(hd)) @ V[i * hkv // hq]
+                    o = np.stack([om.attention_split_lse(q[i], K[i * hkv // hq], V[i * hkv // hq], [(0, n)])
                                   for i in range(hq)])
                     _cmp(f"L{l} attn", og, o)
                 O = st.out(l, "o_proj")
@@ -138,14 +132,14 @@ def test_fullsize_sampled_ops(name):
                     _cmp(f"L{l} q_b", qb, Wt.mv("q_b", l, cqn))
                     kvb = om.dense_matrix(Wt.get("kv_b", l)).reshape(H, nope + vh, kvl)
                     q = qb.reshape(H, nope + rd)
-                    _cmp(f"L{l} absorb", ql, np.einsum("hjc,hj->hc", kvb[:, :nope], R(q[:, :nope])).reshape(-1))
+                    _cmp(f"L{l} absorb", ql, om.mla_absorb_query(R(q[:, :nope]), kvb[:, :nope]).reshape(-1))
                     nl = L * n * kvl
                     C = kv[:nl].reshape(L, n, kvl)[l]
                     PE = kv[nl:].reshape(L, n, rd)[l]
                     qpe = R(rope(q[:, nope:], p, th))
-                    s = (R(ql.reshape(H, kvl)) @ C.T + qpe @ PE.T) / math.sqrt(nope + rd)
-                    _cmp(f"L{l} mla_attn", olat, softmax(s, axis=1) @ C)
-                    _cmp(f"L{l} uv", uv, np.einsum("hvc,hc->hv", kvb[:, nope:], R(olat)).reshape(-1))
+                    olat_ref = om.mla_latent_attention(R(ql.reshape(H, kvl)), qpe, C, PE, 1.0 / math.sqrt(nope + rd))
+                    _cmp(f"L{l} mla_attn", olat, olat_ref)
+                    _cmp(f"L{l} uv", uv, om.mla_up_value(R(olat), kvb[:, nope:]).reshape(-1))
                     _cmp(f"L{l} o_proj", O, Wt.mv("wo", l, R(uv)))
             h = h + O
             m = R(rmsnorm(h, Wt.vector("ffn_norm", l), eps))
@@ -158,22 +152,29 @@ def test_fullsize_sampled_ops(name):
                 else:
                     r = st.out(l, "router")
                     _cmp(f"L{l} router", r, Wt.mv("router", l, m))
-                    idx, _ = om.route_topk(r, w["top_k"])
+                    idx, wts = om.route_topk(r, w["top_k"])
                     got = st.routes.reshape(-1, w["top_k"])[moe_l]
                     if not np.array_equal(got, idx):
                         assert margin_topk(r, w["top_k"]) < 1e-4, f"L{l}: routes {got} vs {idx}"
+                    # gate|up rows: the shared expert's first, then routed slot j's
                     eh, gu, ref = w["expert_hidden"], st.out(l, "exp_gate|up"), []
+                    ns = 1 if w["n_shared"] else 0
+                    if ns:
+                        ref += [Wt.mv("sh_gate", l, m), Wt.mv("sh_up", l, m)]
                     for e in got:
                         ref += [Wt.mv("exp_gate", l, m, int(e)), Wt.mv("exp_up", l, m, int(e))]
-                    if w["n_shared"]:
-                        ref += [Wt.mv("sh_gate", l, m), Wt.mv("sh_up", l, m)]
                     _cmp(f"L{l} experts gate|up", gu, np.concatenate(ref))
-                    dn, ref = st.out(l, "exp_down"), []
-                    for j, e in enumerate(list(got) + ([-1] if w["n_shared"] else [])):
-                        g_, u_ = gu[2 * j * eh:(2 * j + 1) * eh], gu[(2 * j + 1) * eh:(2 * j + 2) * eh]
-                        nm = ("sh_down", -1) if e < 0 else ("exp_down", int(e))
-                        ref.append(Wt.mv(nm[0], l, R(silu(g_) * u_), nm[1]))
-                    _cmp(f"L{l} experts down", dn, np.concatenate(ref))
+                    # the layer's FFN output: routed experts weighted by the GPU's router weights
+                    # (renormalised softmax of its logits), plus the shared expert
+                    ref = np.zeros(d)
+                    gsl = lambda j: (gu[2 * j * eh:(2 * j + 1) * eh], gu[(2 * j + 1) * eh:(2 * j + 2) * eh])
+                    if ns:
+                        g_, u_ = gsl(0)
+                        ref += Wt.mv("sh_down", l, R(silu(g_) * u_))
+                    for j, e in enumerate(got):
+                        g_, u_ = gsl(ns + j)
+                        ref += wts[j] * Wt.mv("exp_down", l, R(silu(g_) * u_), int(e))
+                    _cmp(f"L{l} experts down", st.out(l, "exp_down"), ref)
             if w["arch"] != "dense" and l >= w["n_dense_layers"]:
                 moe_l += 1
             h = h + _ffn_out(st, w, l, moe_l)
@@ -181,37 +182,6 @@ def test_fullsize_sampled_ops(name):
         _cmp("lm_head", st.logits.astype(np.float64), z)
         if margin_topk(z, 1) >= 1e-4:
             assert st.next == argmax_first(z)
-        if name == "dense_gqa_bf16_1k":
-            # End to end, this random-init 16-layer bf16 model is chaotic: one bf16-ulp change of a
-            # single activation element in layer 0 moves the oracle's own logits by ~1e-2 of max|z|.
-            # The GPU must stay within twice that single-flip sensitivity, measured here, and agree on
-            # the greedy token wherever the oracle's margin exceeds that band.
-            cache = om.synthetic_cache(w)
-            od = om.OracleDecoder(w, Wt)
-            od.set_cache(cache, w["ctx"])
-            ref = od.step(st.first)
-            orig, calls = om.gemv, [0]
-
-            def flip_one(t, x):
-                calls[0] += 1
-                if calls[0] == 1:  # first GEMV input of layer 0: one element up by one bf16 ulp
-                    x = x.copy()
-                    x[7] += abs(x[7]) * 2.0 ** -8
-                return orig(t, x)
-
-            om.gemv = flip_one
-            try:
-                od2 = om.OracleDecoder(w, Wt)
-                od2.set_cache(cache, w["ctx"])
-                flipped = od2.step(st.first)["logits"]
-            finally:
-                om.gemv = orig
-            zmax = np.max(np.abs(ref["logits"]))
-            band = 2.0 * np.max(np.abs(flipped - ref["logits"]))
-            e2e = np.max(np.abs(st.logits - ref["logits"]))
-            assert e2e <= band, f"end-to-end logits differ by {e2e / zmax:.3e} of max|z|, band {band / zmax:.3e}"
-            if margin_topk(ref["logits"], 1) > 2 * band:
-                assert st.next == ref["next"]
     finally:
         st.close()
         torch.cuda.empty_cache()

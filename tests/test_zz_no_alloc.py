@@ -11,6 +11,15 @@ q/k/v output and the KV cache after the new row was appended) and its output
 (the split-KV partials, combined here); the allocation-free call on the same
 inputs must agree within the bf16 tolerance of the other GPU tests.
 
+A second set of cases checks the call against the oracle's float64 attention
+(the split-KV definition taken as one chunk, softmax(q K^T / sqrt(head_dim)) V) on
+seeded random q and bf16 K/V, over shapes the decode step never produces: head_dim
+128 with 8 query heads per kv head, a cache row stride larger than the positions
+used, one position, thousands of positions (many shared-memory tiles per chunk, so
+the online softmax rescales across tiles), and 64 chunks on a single kv head.  The
+host-side refusals (unsupported shapes, misaligned pointers, partials larger than
+the fixed scratch) return before anything is launched.
+
 Kept in its own file, collected last, so a run that stops at the first failure
 has run every other test before it.
 """
@@ -18,6 +27,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import model as om
 from synth import device as sdev
 from synth import workloads
 
@@ -46,14 +56,13 @@ def test_noalloc_attention_matches_decode_step():
         d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
         plan = [line.split() for line in d.plan_text().splitlines()[:-1]]
         assert plan[0][1] == "qkv" and plan[1][1] == "attn"
-        S = int(dict(f.split("=") for f in plan[0][2:] if "=" in f)["S"])
         nch = int(dict(f.split("=") for f in plan[1][2:] if "=" in f)["nch"])
         tok = 5
         for call in range(2):
             pos = w["ctx"] + call
             tok = d.step(tok)
             # the step's attention inputs: q of layer 0 (RoPE at pos, rounded to bf16) ...
-            qkv = np.frombuffer(d.dump(pkg.dec.DEC_DUMP_OP + 0), np.float32).astype(np.float64).reshape(S, -1).sum(0)
+            qkv = np.frombuffer(d.dump(pkg.dec.DEC_DUMP_OP + 0), np.float32).astype(np.float64)
             qr = qkv[: hq * hd].reshape(hq, hd)
             half = hd // 2
             ang = pos * w["rope_theta"] ** (-2.0 * np.arange(half) / hd)
@@ -88,6 +97,41 @@ def test_noalloc_attention_matches_decode_step():
         d.close()
 
 
+ORACLE_TOL = 1e-4  # fp32 GPU arithmetic against float64 on the same bf16 / fp32 inputs
+
+# (n_heads, n_kv_heads, head_dim, n_pos, cache_stride)
+SHAPES = [(6, 2, 64, 79, 79), (16, 2, 128, 3000, 4096), (8, 8, 128, 1, 16), (32, 8, 64, 1025, 2048),
+          (8, 1, 64, 5000, 5000)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "h%d_kv%d_d%d_n%d_s%d" % s)
+def test_noalloc_attention_matches_oracle(shape):
+    import persistent_sm_decode_02_b200 as pkg
+
+    hq, hkv, hd, n, stride = shape
+    rng = np.random.default_rng(1000 + hq * 7 + hd + n)
+    kv = torch.from_numpy(rng.standard_normal((2, hkv, stride, hd)).astype(np.float32)).to(torch.bfloat16)
+    kv_d = kv.view(torch.int16).cuda()
+    kv64 = kv.float().numpy().astype(np.float64)
+    out = torch.empty(hq * hd, dtype=torch.float32, device="cuda")
+    gs = hq // hkv
+    for call in range(2):  # two calls in a row share the fixed scratch
+        q = rng.standard_normal((hq, hd)).astype(np.float32)
+        qd = torch.from_numpy(q).cuda()
+        torch.cuda.synchronize()
+        rc = pkg.dec.dec_attention_noalloc(qd.data_ptr(), kv_d[0].data_ptr(), kv_d[1].data_ptr(), hq, hkv, hd, n,
+                                           stride, out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert rc == pkg.dec.DEC_OK
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().astype(np.float64).reshape(hq, hd)
+        ref = np.stack([om.attention_split_lse(q[h].astype(np.float64), kv64[0, h // gs, :n], kv64[1, h // gs, :n],
+                                               [(0, n)]) for h in range(hq)])
+        err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
+        assert err <= ORACLE_TOL, f"call {call}: max error {err:.3e}"
+        if n == 1:  # one position: the output is that position's V row
+            assert np.max(np.abs(got - kv64[1, np.arange(hq) // gs, 0])) <= ORACLE_TOL * np.max(np.abs(ref))
+
+
 def test_noalloc_attention_rejects_bad_shapes():
     import persistent_sm_decode_02_b200 as pkg
 
@@ -97,3 +141,10 @@ def test_noalloc_attention_rejects_bad_shapes():
     assert pkg.dec.dec_attention_noalloc(p, p, p, 4, 4, 96, 4, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
     assert pkg.dec.dec_attention_noalloc(p, p, p, 6, 4, 64, 4, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
     assert pkg.dec.dec_attention_noalloc(p, p, p, 4, 4, 64, 8, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
+    # K / V not 16-byte aligned, q / out not 4-byte aligned (refused before any launch)
+    assert pkg.dec.dec_attention_noalloc(p, p + 2, p, 4, 4, 64, 4, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
+    assert pkg.dec.dec_attention_noalloc(p, p, p + 8, 4, 4, 64, 4, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
+    assert pkg.dec.dec_attention_noalloc(p + 2, p, p, 4, 4, 64, 4, 4, p, None) == pkg.dec.DEC_ERR_INVALID_ARG
+    assert pkg.dec.dec_attention_noalloc(p, p, p, 4, 4, 64, 4, 4, p + 1, None) == pkg.dec.DEC_ERR_INVALID_ARG
+    # one chunk per head already needs 4096 * 130 floats, more than the fixed 2 MiB scratch
+    assert pkg.dec.dec_attention_noalloc(p, p, p, 4096, 512, 128, 4, 4, p, None) == pkg.dec.DEC_ERR_CAPACITY
