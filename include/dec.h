@@ -107,13 +107,13 @@ enum {
                                      first stage (ns; 0 for a task that streams nothing) */
 #define DEC_DUMP_PLAN 4     /* text: one line per op (kind, tasks, geometry) */
 #define DEC_DUMP_WEIGHTS 5  /* bytes of weights read per step (uint64 x2: weights+scales, stored incl. padding) */
-#define DEC_DUMP_STATUS 7   /* int32 x12: device status word {code, cta, op, task} (code 0 ok, 1 timeout,
-                               2 non-finite logit), then the step state {epoch, pos, tok, last, stop, 0, 0, 0} */
+#define DEC_DUMP_STATUS 7   /* 64 bytes: device status word {int32 code, cta, op, task (code 0 ok, 1 timeout,
+                               2 non-finite logit); uint64 winning key of the last final op (logit bits in
+                               order-preserving form << 32 | ~token); uint64 0}, then the step state
+                               {int32 epoch, pos, tok, last, stop, 0, 0, 0} */
 #define DEC_DUMP_OP 100     /* + op index (DEC_DUMP_PLAN order): fp32 outputs of that op in the last step;
-                               GEMV ops: [rows] (ops whose rows add into one accumulator, the routed and
-                               shared experts' down projections, give the same summed vector); attention
-                               ops: max [heads][chunks], sum [heads][chunks], weighted values
-                               [heads][chunks][dim], concatenated */
+                               GEMV ops: partial sums [splits][rows]; attention ops: max [heads][chunks],
+                               sum [heads][chunks], weighted values [heads][chunks][dim], concatenated */
 
 /* ------------------------------------------------------------------ types */
 typedef struct dec_ctx dec_ctx; /* opaque; owns all of its device memory */

@@ -32,7 +32,7 @@ namespace {
 // A weight matrix stored in tile order: [row tile][split][stage][R][kcb bytes].
 struct Mat {
   int N = 0, K = 0, wb = 1, wtype = WT_F32;
-  int R = 0, nst = 1, kcb = 0, Kpad = 0, ntiles = 0;  // nst: stages per row tile
+  int R = 0, S = 1, nst = 1, kcb = 0, Kpad = 0, ntiles = 0;
   int n_experts = 1;
   int mode = 0;  // source layout: 0 row-major [N][K]; 1 W_UK^T of kv_b; 2 W_UV of kv_b
   size_t tile_bytes = 0;  // bytes of one expert
@@ -58,9 +58,9 @@ Geo gemv_geometry(int K, int wb) {
   int best = -1;
   long long best_waste = 1LL << 62;
   // Prefer 512-byte row chunks: 32 lanes cover a row, so every row reduces
-  // inside one warp and tasks need no CTA-wide barrier; narrower chunks only when
+  // inside one warp and tasks need no CTA-wide barrier; wider chunks only when
   // 512 would pad K too much.
-  for (int kcb = 512; kcb >= 64; kcb >>= 1) {  // the widths the kernels are compiled for
+  for (int kcb = 512; kcb >= 32; kcb >>= 1) {
     const long long pad = (Kb + kcb - 1) / kcb * kcb;
     const long long waste = pad - Kb;
     if (waste * 16 <= Kb) {
@@ -83,9 +83,32 @@ Geo gemv_geometry(int K, int wb) {
   return g;
 }
 
-__global__ void relayout16(const uint8_t* src, long long N, long long K, int wb, int R, int nst, int kcb,
+// Split-K factor S of a GEMV op, in units of ring stages on the busiest CTA: its tasks'
+// stages plus a fixed cost per task, plus the consumer's prologue, which reads all S
+// partial vectors (out_rows fp32 values each) on every CTA.  Every CTA reads the same lines
+// at once, and that L2 read ran about 4x slower per byte than a weight stage in the device
+// trace, hence the weight.
+constexpr double kPrologueWeight = 4.0;
+int choose_split(int ntiles, int nst_total, int n_ctas, long long out_rows, bool force_one) {
+  if (force_one) return 1;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int S = 1; S <= 16 && S <= nst_total; ++S) {
+    if (nst_total % S) continue;
+    const long long tasks = (long long)ntiles * S;
+    const long long per = (tasks + n_ctas - 1) / n_ctas;
+    const double cost = per * (nst_total / (double)S + 0.75) + kPrologueWeight * S * out_rows * 4.0 / kStageBytes;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+__global__ void relayout16(const uint8_t* src, long long N, long long K, int wb, int R, int S, int nst, int kcb,
                            long long total16, uint8_t* dst) {
-  // dst byte q = (((rt*nst + st)*R + r)*kcb + jb); one thread per 16 bytes
+  // dst byte q = ((((rt*S + s)*nst + st)*R + r)*kcb + jb); one thread per 16 bytes
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total16;
        i += (long long)gridDim.x * blockDim.x) {
     const long long q = i * 16;
@@ -94,9 +117,11 @@ __global__ void relayout16(const uint8_t* src, long long N, long long K, int wb,
     const long long r = rest % R;
     rest /= R;
     const long long st = rest % nst;
-    const long long rt = rest / nst;
+    rest /= nst;
+    const long long s = rest % S;
+    const long long rt = rest / S;
     const long long n = rt * R + r;
-    const long long kb = st * kcb + jb;  // byte offset in the padded row
+    const long long kb = (s * nst + st) * kcb + jb;  // byte offset in the padded row
     uint4 v = make_uint4(0, 0, 0, 0);
     if (n < N && kb < K * wb) v = *reinterpret_cast<const uint4*>(src + n * K * wb + kb);
     *reinterpret_cast<uint4*>(dst + q) = v;
@@ -104,7 +129,7 @@ __global__ void relayout16(const uint8_t* src, long long N, long long K, int wb,
 }
 
 // Element-wise re-layout for the two views of kv_b (mode 1: W_UK^T, mode 2: W_UV).
-__global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long long K, int wb, int R, int nst,
+__global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long long K, int wb, int R, int S, int nst,
                              int kcb, long long total, int nope, int vdim, int kvl, uint8_t* dst) {
   for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < total;
        q += (long long)gridDim.x * blockDim.x) {
@@ -113,9 +138,11 @@ __global__ void relayout_kvb(const uint8_t* src, int mode, long long N, long lon
     const long long r = rest % R;
     rest /= R;
     const long long st = rest % nst;
-    const long long rt = rest / nst;
+    rest /= nst;
+    const long long s = rest % S;
+    const long long rt = rest / S;
     const long long n = rt * R + r;
-    const long long kb = st * kcb + jb;
+    const long long kb = (s * nst + st) * kcb + jb;
     const long long k = kb / wb, byte = kb % wb;
     uint8_t v = 0;
     if (n < N && k < K) {
@@ -173,6 +200,9 @@ struct dec_ctx {
   std::vector<OpDesc> ops;
   std::vector<std::string> op_names;
   OpDesc* d_ops = nullptr;
+  int2* d_tasks = nullptr;
+  int* d_task_off = nullptr;
+  std::vector<int> task_off;
   int lm_op = -1, final_op = -1;
   // memory
   std::vector<void*> allocs;
@@ -205,9 +235,6 @@ struct dec_ctx {
   cudaGraphExec_t graph = nullptr;
   int mode = DEC_PERSISTENT;
   std::vector<std::vector<void*>> seg_mats;  // per op: the Mat behind every segment
-  unsigned* d_cursors = nullptr;             // task cursors [2][n_cursors]
-  int n_cursors = 0;
-  std::vector<std::pair<void*, size_t>> accs;  // fixed-point accumulators, cleared by dec_reset
   uint8_t* staging = nullptr;
   size_t staging_bytes = 0;
   void* kvb_src = nullptr;
@@ -280,7 +307,6 @@ struct Planner {
     o.layer = layer;
     o.dep[0] = o.dep[1] = -1;
     o.pdep = -1;
-    o.ngroups = 1;
     o.in_bf16 = c->act_bf16;
     o.eps = c->cfg.norm_eps;
     return o;
@@ -298,18 +324,18 @@ struct Planner {
   }
 
   // Create a GEMV op over segments sharing K; returns op index.
-  // A row tile of more than kPieceStages ring stages is cut along K into equal pieces
-  // (one task each) that add into a fixed-point accumulator (dec_types.h), so tasks
-  // stay short and the run-time task hand-out can balance the SMs; whole_tiles keeps
-  // one task per tile with an fp32 output row (the LM head's argmax keys, absorb_q's
-  // bf16 query, ops grouped per head).  same_rows: every segment adds into the same
-  // output rows (the experts' down projections, the routed ones weighted by the router),
-  // which also needs the accumulator.  Segments that read different input groups get
-  // one task cursor each.
-  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool whole_tiles, const char* name,
-           bool same_rows = false, bool fp32_out = false) {
+  // whole_reader: every CTA running the consumer reads the whole output (a GEMV prologue);
+  // false when each consumer task reads only its own slice (attention reading q/k/v).
+  int gemv(const std::vector<SegSpec>& segs, int K, int layer, bool force_s1, const char* name,
+           bool whole_reader = true) {
     OpDesc o = base_op(OP_GEMV, layer);
     const Geo g = gemv_geometry(K, c->wb);
+    int ntiles = 0;
+    for (auto& s : segs) ntiles += (s.mat->N + g.R - 1) / g.R;
+    long long out_rows = 0;
+    if (whole_reader)
+      for (auto& sp : segs) out_rows += sp.mat->N;
+    const int S = choose_split(ntiles, g.nst_total, c->n_ctas, out_rows, force_s1);
     o.wtype = c->wtype;
     o.K = K;
     o.Kpad = g.Kpad;
@@ -319,28 +345,24 @@ struct Planner {
     o.G = g.G;
     o.rpt = g.rpt;
     o.R = g.R;
-    o.nst_total = g.nst_total;
+    o.S = S;
+    o.nst = g.nst_total / S;
     o.n = K;
     o.nsegs = (int)segs.size();
     if (o.nsegs > kMaxSegs) {
       rc = fail(c, DEC_ERR_UNSUPPORTED, "too many segments in %s", name);
       return -1;
     }
-    const int nps = whole_tiles ? 1 : (g.nst_total + kPieceStages - 1) / kPieceStages;  // pieces per tile
-    const bool acc = nps > 1 || same_rows;  // tasks add into rows (else one task stores each row)
-    bool groups = false;
-    for (auto& sp : segs) groups |= sp.in_group != segs[0].in_group;
     int task = 0, out = 0;
-    std::vector<int4> pieces;
-    std::vector<int> gb;
     for (int i = 0; i < o.nsegs; ++i) {
       Mat* m = segs[i].mat;
       m->R = g.R;
-      m->nst = g.nst_total;
+      m->S = S;
+      m->nst = o.nst;
       m->kcb = g.kcb;
       m->Kpad = g.Kpad;
       m->ntiles = (m->N + g.R - 1) / g.R;
-      m->tile_bytes = (size_t)m->ntiles * g.nst_total * g.R * g.kcb;
+      m->tile_bytes = (size_t)m->ntiles * S * o.nst * g.R * g.kcb;
       m->sc_count = c->wtype == WT_FP8 ? (size_t)((m->N + 127) / 128) * ((m->K + 127) / 128) : 0;
       Seg& sg = o.seg[i];
       sg.slot = segs[i].slot;
@@ -348,48 +370,15 @@ struct Planner {
       sg.N = m->N;
       sg.ntiles = m->ntiles;
       sg.task0 = task;
-      sg.out_off = same_rows ? 0 : out;
+      sg.out_off = out;
       sg.w_estride = (long long)m->tile_bytes;
       sg.s_estride = (long long)m->sc_count;
-      sg.zero_acc = acc && (!same_rows || i == 0);
-      if (groups) gb.push_back(acc ? (int)pieces.size() : task);
-      if (acc)
-        for (int r = 0; r < m->ntiles; ++r)
-          for (int p = 0; p < nps; ++p) {
-            const int a = p * g.nst_total / nps, b = (p + 1) * g.nst_total / nps;
-            pieces.push_back(make_int4(i, r, a, b - a));
-          }
-      task += m->ntiles;
-      if (!same_rows || i == 0) out += m->N;
+      task += m->ntiles * S;
+      out += m->N;
     }
+    o.ntasks = task;
     o.out_stride = out;
-    int arc = DEC_OK;
-    if (fp32_out) {
-      arc = dalloc(c, &o.out, (size_t)o.out_stride * 4);
-    } else if (!(arc = dalloc(c, &o.acc, (size_t)2 * o.out_stride * 8))) {
-      c->accs.push_back({o.acc, (size_t)2 * o.out_stride * 8});
-      o.acc_add = acc ? 1 : 0;
-    }
-    if (arc) {
-    } else if (!acc) {
-      o.ntasks = task;
-    } else {
-      o.ntasks = (int)pieces.size();
-      int4* dp = nullptr;
-      if (!(arc = dalloc(c, &dp, pieces.size() * sizeof(int4))) &&
-          cudaMemcpy(dp, pieces.data(), pieces.size() * sizeof(int4), cudaMemcpyHostToDevice) != cudaSuccess)
-        arc = fail(c, DEC_ERR_CUDA, "piece table of %s", name);
-      o.pieces = dp;
-    }
-    if (!arc && groups) {
-      gb.push_back(o.ntasks);
-      o.ngroups = (int)gb.size() - 1;
-      int* dg = nullptr;
-      if (!(arc = dalloc(c, &dg, gb.size() * sizeof(int))) &&
-          cudaMemcpy(dg, gb.data(), gb.size() * sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
-        arc = fail(c, DEC_ERR_CUDA, "task groups of %s", name);
-      o.gbegin = dg;
-    }
+    int arc = dalloc(c, &o.out, (size_t)o.S * o.out_stride * 4);
     if (arc) {
       rc = arc;
       return -1;
@@ -434,7 +423,7 @@ static size_t mla_cache_bytes(const dec_config& f) {
 // Grouped GEMVs whose row tiles are tiny (absorb_q: 16 KB, uv: 32 KB per tile) run a whole
 // input group (one head) per task: the prologue and the task overhead are paid once per head.
 static void group_tasks(OpDesc& o) {
-  if (o.kind != OP_GEMV || o.pieces || o.rows_per_group <= 0 || o.rows_per_group % o.R) return;
+  if (o.kind != OP_GEMV || o.S != 1 || o.rows_per_group <= 0 || o.rows_per_group % o.R) return;
   const int tpt = o.rows_per_group / o.R;
   if (tpt <= 1 || o.ntasks % tpt) return;
   for (int i = 0; i < o.nsegs; ++i)
@@ -445,9 +434,6 @@ static void group_tasks(OpDesc& o) {
 
 static float* gainp(dec_ctx* c, int kind, int layer) { return c->vecs[{kind, layer}].p; }
 
-// The output of GEMV op o from element `off` on, as its consumers read it.
-static PSet out_of(const OpDesc& o, int off = 0) { return PSet{o.acc, o.out_stride, off}; }
-
 static int build_plan(dec_ctx* c) {
   const dec_config& f = c->cfg;
   Planner P{c};
@@ -456,8 +442,9 @@ static int build_plan(dec_ctx* c) {
   const bool mla = f.arch == DEC_ARCH_MLA_MOE;
   // per-layer bookkeeping of the ops whose outputs feed the next layer's residual
   struct LayerOut {
-    int ffn_op = -1;   // dense down op, or the MoE layer's routed expert-down op
-    int ffn_op2 = -1;  // MoE: the shared expert's down op (adds into the same accumulator)
+    int ffn_op = -1;        // dense down op or MoE expert-down op
+    int router_op = -1;     // MoE router op
+    int mid_buf = -1;
   };
   std::vector<LayerOut> lo(L);
   std::vector<float*> h_in(L), h_mid(L);
@@ -478,10 +465,22 @@ static int build_plan(dec_ctx* c) {
       o.embed_bf16 = c->act_bf16;
     } else {
       const LayerOut& p = lo[l - 1];
+      const OpDesc& fo = c->ops[p.ffn_op];
       o.h_base = h_mid[l - 1];
-      o.add = out_of(c->ops[p.ffn_op]);
-      o.dep[0] = p.ffn_op;
-      o.dep[1] = p.ffn_op2;
+      if (p.router_op < 0) {
+        o.add = PSet{fo.out, fo.S, fo.out_stride, 0};
+        o.dep[0] = p.ffn_op;
+      } else {
+        const OpDesc& ro = c->ops[p.router_op];
+        o.routed = PSet{fo.out, fo.S, fo.out_stride, 0};
+        o.routed_slot_stride = d;
+        o.rt_w = ro.rt_w;
+        o.n_experts = f.n_experts;
+        o.top_k = f.top_k;
+        if (f.n_shared > 0) o.add2 = PSet{fo.out, fo.S, fo.out_stride, f.top_k * d};
+        o.dep[0] = p.ffn_op;
+        o.dep[1] = p.router_op;
+      }
     }
   };
 
@@ -501,7 +500,7 @@ static int build_plan(dec_ctx* c) {
       Mat* wq = P.new_mat(DEC_W_Q, l, hq * hd, d, 1, 0);
       Mat* wk = P.new_mat(DEC_W_K, l, hkv * hd, d, 1, 0);
       Mat* wv = P.new_mat(DEC_W_V, l, hkv * hd, d, 1, 0);
-      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv");
+      int qkv = P.gemv({{wq, -1, 0}, {wk, -1, 0}, {wv, -1, 0}}, d, l, false, "qkv", false);
       if (qkv < 0) return P.rc;
       {
         OpDesc& o = c->ops[qkv];
@@ -515,7 +514,8 @@ static int build_plan(dec_ctx* c) {
       a.hd = hd;
       a.gs = hq / hkv;
       {
-        a.qkv = out_of(c->ops[qkv]);
+        const OpDesc& p = c->ops[qkv];
+        a.qkv = PSet{p.out, p.S, p.out_stride, 0};
       }
       a.nch = nch_dense;
       a.ntasks = hkv * a.nch;
@@ -532,7 +532,7 @@ static int build_plan(dec_ctx* c) {
       a.m_out = attn_buf[0];
       a.l_out = attn_buf[1];
       a.o_out = attn_buf[2];
-      if (dalloc(c, &a.o_fin, (size_t)2 * hq * hd * 8)) return DEC_ERR_OOM;
+      if (dalloc(c, &a.o_fin, (size_t)hq * hd * 4)) return DEC_ERR_OOM;
       a.kcache = c->kc[l];
       a.vcache = c->vc[l];
       a.rope_cos = c->rope_cos;
@@ -544,7 +544,7 @@ static int build_plan(dec_ctx* c) {
       OpDesc& oo = c->ops[o_op];
       oo.pro = PRO_SUM;  // the attention op's last chunk task per kv head combined the chunks
       oo.n = hq * hd;
-      oo.src = PSet{c->ops[attn].o_fin, hq * hd, 0};
+      oo.src = PSet{c->ops[attn].o_fin, 1, hq * hd, 0};
       oo.dep[0] = attn;
     } else {
       const int H = f.n_heads, nope = f.qk_nope, rd = f.qk_rope, vh = f.v_head, kvl = f.kv_lora;
@@ -558,14 +558,15 @@ static int build_plan(dec_ctx* c) {
         o.h_out = h_in[l];
       }
       Mat* qb = P.new_mat(DEC_W_Q_B, l, H * (nope + rd), f.q_lora, 1, 0);
-      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b");
+      int s2 = P.gemv({{qb, -1, 0}}, f.q_lora, l, false, "q_b", false);  // absorb_q reads one head per task
       if (s2 < 0) return P.rc;
       {
         OpDesc& o = c->ops[s2];
+        const OpDesc& p = c->ops[s1];
         o.pro = PRO_NORM_SUM;
         o.n = f.q_lora;
         o.gain = gainp(c, DEC_W_Q_A_NORM, l);
-        o.src = out_of(c->ops[s1]);
+        o.src = PSet{p.out, p.S, p.out_stride, 0};
         o.dep[0] = s1;
       }
       Mat* uk = P.new_mat(DEC_W_KV_B * 16 + 1, l, H * kvl, nope, 1, 1);  // W_UK^T view of kv_b
@@ -580,9 +581,10 @@ static int build_plan(dec_ctx* c) {
       }
       {
         OpDesc& o = c->ops[s3];
+        const OpDesc& p = c->ops[s2];
         o.pro = PRO_SUM;
         o.n = nope;
-        o.src = out_of(c->ops[s2]);
+        o.src = PSet{p.out, p.S, p.out_stride, 0};
         o.gstride = nope + rd;
         o.rows_per_group = kvl;
         o.dep[0] = s2;
@@ -592,7 +594,8 @@ static int build_plan(dec_ctx* c) {
         o.rope_cos = c->rope_cos;
         o.rope_sin = c->rope_sin;
         // an extra last task appends the step's latent row (normalised c, RoPE'd k_pe) to the cache
-        o.ckv = out_of(c->ops[s1], f.q_lora);
+        const OpDesc& p1 = c->ops[s1];
+        o.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
         o.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
         o.kcache = c->kc[l];
         group_tasks(o);
@@ -600,6 +603,7 @@ static int build_plan(dec_ctx* c) {
       }
       OpDesc a = P.base_op(OP_MLA, l);
       {
+        const OpDesc& p1 = c->ops[s1];
         a.H = H;
         a.kvl = kvl;
         a.rdim = rd;
@@ -607,7 +611,7 @@ static int build_plan(dec_ctx* c) {
         a.nch = nch_mla;
         a.ntasks = nch_mla;
         a.qc = qc;
-        a.ckv = out_of(c->ops[s1], f.q_lora);
+        a.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};
         a.dep[0] = s3;
         a.pdep = s3;  // the producer streams the absorbed query
         a.max_seq = f.max_seq;
@@ -629,7 +633,7 @@ static int build_plan(dec_ctx* c) {
       a.kvnorm_g = gainp(c, DEC_W_KV_A_NORM, l);
       const int attn = P.push(a, "mla_attn");
       Mat* uv = P.new_mat(DEC_W_KV_B * 16 + 2, l, H * vh, kvl, 1, 2);  // W_UV view of kv_b
-      int s5 = P.gemv({{uv, -1, -1}}, kvl, l, true, "uv");
+      int s5 = P.gemv({{uv, -1, -1}}, kvl, l, false, "uv");
       if (s5 < 0) return P.rc;
       {
         OpDesc& o = c->ops[s5];
@@ -650,14 +654,16 @@ static int build_plan(dec_ctx* c) {
       if (o_op < 0) return P.rc;
       {
         OpDesc& o = c->ops[o_op];
+        const OpDesc& p = c->ops[s5];
         o.pro = PRO_SUM;
         o.n = H * vh;
-        o.src = out_of(c->ops[s5]);
+        o.src = PSet{p.out, p.S, p.out_stride, 0};
         o.dep[0] = s5;
       }
     }
     // ---- FFN
-    const PSet o_out = out_of(c->ops[o_op]);
+    const OpDesc& oo = c->ops[o_op];
+    const PSet o_out{oo.out, oo.S, oo.out_stride, 0};
     auto ffn_resid = [&](OpDesc& o, bool write_h) {
       o.pro = PRO_RESID_NORM;
       o.n = d;
@@ -679,10 +685,11 @@ static int build_plan(dec_ctx* c) {
       if (dn < 0) return P.rc;
       {
         OpDesc& o = c->ops[dn];
+        const OpDesc& p = c->ops[gu];
         o.pro = PRO_SWIGLU;
         o.n = ff;
-        o.gate = out_of(c->ops[gu]);
-        o.up = out_of(c->ops[gu], ff);
+        o.gate = PSet{p.out, p.S, p.out_stride, 0};
+        o.up = PSet{p.out, p.S, p.out_stride, ff};
         o.slot_stride = 0;
         o.dep[0] = gu;
       }
@@ -702,31 +709,24 @@ static int build_plan(dec_ctx* c) {
         CK(cudaMemsetAsync(o.rt_ids, 0, (size_t)k * 4, c->stream));
         CK(cudaMemsetAsync(o.rt_w, 0, (size_t)k * 4, c->stream));
       }
-      int* rids = c->ops[ro].rt_ids;
-      float* rw = c->ops[ro].rt_w;
-      // The shared expert's segments come first: its weights do not wait for the router, so
-      // the first tasks handed out stream while the router's top-k is decided.  Input group
-      // 0 is the shared expert's SwiGLU input, group j + 1 routed slot j's.
       Mat* eg = P.new_mat(DEC_W_EXP_GATE, l, eh, d, E, 0);
       Mat* eu = P.new_mat(DEC_W_EXP_UP, l, eh, d, E, 0);
-      Mat* ed = P.new_mat(DEC_W_EXP_DOWN, l, d, eh, E, 0);
-      std::vector<SegSpec> segs, dsegs;
-      const int g0 = f.n_shared > 0 ? 1 : 0;  // group of routed slot 0
-      if (f.n_shared > 0) {
-        Mat* sg = P.new_mat(DEC_W_SH_GATE, l, eh * f.n_shared, d, 1, 0);
-        Mat* su = P.new_mat(DEC_W_SH_UP, l, eh * f.n_shared, d, 1, 0);
-        Mat* sd = P.new_mat(DEC_W_SH_DOWN, l, d, eh * f.n_shared, 1, 0);
-        segs.push_back({sg, -1, 0});
-        segs.push_back({su, -1, 0});
-        dsegs.push_back({sd, -1, 0});
-      }
+      Mat* sg = nullptr;
+      Mat* su = nullptr;
+      std::vector<SegSpec> segs;
       for (int j = 0; j < k; ++j) {
         segs.push_back({eg, j, 0});
         segs.push_back({eu, j, 0});
-        dsegs.push_back({ed, j, g0 + j});
+      }
+      if (f.n_shared > 0) {
+        sg = P.new_mat(DEC_W_SH_GATE, l, eh * f.n_shared, d, 1, 0);
+        su = P.new_mat(DEC_W_SH_UP, l, eh * f.n_shared, d, 1, 0);
+        segs.push_back({sg, -1, 0});
+        segs.push_back({su, -1, 0});
       }
       int egu = P.gemv(segs, d, l, false, "exp_gate|up");
       if (egu < 0) return P.rc;
+      int* rids = c->ops[ro].rt_ids;
       {
         OpDesc& o = c->ops[egu];
         ffn_resid(o, false);
@@ -735,30 +735,38 @@ static int build_plan(dec_ctx* c) {
         o.n_experts = E;
         o.top_k = k;
       }
-      int edn = P.gemv(dsegs, eh, l, false, "exp_down", true);
+      Mat* ed = P.new_mat(DEC_W_EXP_DOWN, l, d, eh, E, 0);
+      Mat* sd = nullptr;
+      std::vector<SegSpec> dsegs;
+      for (int j = 0; j < k; ++j) dsegs.push_back({ed, j, j});
+      if (f.n_shared > 0) {
+        sd = P.new_mat(DEC_W_SH_DOWN, l, d, eh * f.n_shared, 1, 0);
+        dsegs.push_back({sd, -1, k});
+      }
+      int edn = P.gemv(dsegs, eh, l, false, "exp_down");
       if (edn < 0) return P.rc;
       {
         OpDesc& o = c->ops[edn];
+        const OpDesc& p = c->ops[egu];
         o.pro = PRO_SWIGLU;
         o.n = eh;
-        o.gate = out_of(c->ops[egu]);
-        o.up = out_of(c->ops[egu], eh);
+        o.gate = PSet{p.out, p.S, p.out_stride, 0};
+        o.up = PSet{p.out, p.S, p.out_stride, eh};
         o.slot_stride = 2 * eh;
         o.dep[0] = egu;
-        o.dep[1] = ro;  // the slot weights it applies
         o.pdep = ro;
         o.rt_ids = rids;
-        o.rt_w = rw;
         o.n_experts = E;
         o.top_k = k;
       }
       lo[l].ffn_op = edn;
+      lo[l].router_op = ro;
       ++c->n_moe;
     }
   }
   // ---- LM head + argmax
   Mat* lm = P.new_mat(DEC_W_LM_HEAD, -1, V, d, 1, 0);
-  int lmop = P.gemv({{lm, -1, 0}}, d, -1, true, "lm_head", false, true);
+  int lmop = P.gemv({{lm, -1, 0}}, d, -1, true, "lm_head");
   if (lmop < 0) return P.rc;
   {
     OpDesc& o = c->ops[lmop];
@@ -784,21 +792,34 @@ static int build_plan(dec_ctx* c) {
   return DEC_OK;
 }
 
-// ---------------------------------------------------------- task cursors
-// Every op gets one cursor per task group (two copies, for alternate steps), and its
-// first record in the trace buffer.
-static int setup_cursors(dec_ctx* c) {
-  int ncur = 0, trace = 0;
-  for (auto& o : c->ops) {
-    if (o.ngroups < 1) o.ngroups = 1;
-    o.cur_off = ncur;
-    o.trace_base = trace;
-    ncur += o.ngroups;
-    trace += o.ntasks;
+// ---------------------------------------------------------- task lists
+// Each op's tasks are cut into n_ctas contiguous runs, one per CTA, starting
+// at a CTA that rotates from op to op so that the remainders spread evenly.
+// Contiguous runs keep a CTA on one input group (expert slot, head) so that
+// the prologue building that group's input runs once per CTA, not per task.
+static int assign_tasks(dec_ctx* c) {
+  std::vector<std::vector<int2>> lists(c->n_ctas);
+  const int nc = c->n_ctas;
+  int rr = 0;
+  for (int op = 0; op < (int)c->ops.size(); ++op) {
+    const long long n = c->ops[op].ntasks;
+    for (int i = 0; i < nc; ++i) {
+      const int b = (rr + i) % nc;
+      for (long long t = i * n / nc; t < (i + 1) * n / nc; ++t) lists[b].push_back(make_int2(op, (int)t));
+    }
+    rr = (int)((rr + n) % nc);
   }
-  c->n_cursors = ncur;
-  if (dalloc(c, &c->d_cursors, (size_t)2 * ncur * 4)) return DEC_ERR_OOM;
-  c->accs.push_back({c->d_cursors, (size_t)2 * ncur * 4});  // cleared with the accumulators
+  std::vector<int2> flat;
+  c->task_off.assign(c->n_ctas + 1, 0);
+  for (int b = 0; b < c->n_ctas; ++b) {
+    c->task_off[b] = (int)flat.size();
+    flat.insert(flat.end(), lists[b].begin(), lists[b].end());
+  }
+  c->task_off[c->n_ctas] = (int)flat.size();
+  if (dalloc(c, &c->d_tasks, flat.size() * sizeof(int2))) return DEC_ERR_OOM;
+  if (dalloc(c, &c->d_task_off, c->task_off.size() * sizeof(int))) return DEC_ERR_OOM;
+  CK(cudaMemcpy(c->d_tasks, flat.data(), flat.size() * sizeof(int2), cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(c->d_task_off, c->task_off.data(), c->task_off.size() * sizeof(int), cudaMemcpyHostToDevice));
   return DEC_OK;
 }
 
@@ -862,7 +883,7 @@ static int validate(const dec_config* f, dec_ctx* c) {
 static int check_work_area(dec_ctx* c) {
   // The prologues read partial sums with 16-byte loads: every vector they read
   // must start, and every split must be strided, at a multiple of 4 floats.
-  auto al = [](const PSet& p) { return !p.acc || (p.off % 4 == 0 && p.stride % 4 == 0); };
+  auto al = [](const PSet& p) { return !p.ptr || (p.off % 4 == 0 && p.stride % 4 == 0); };
   for (size_t i = 0; i < c->ops.size(); ++i) {
     const OpDesc& o = c->ops[i];
     const char* nm = c->op_names[i].c_str();
@@ -870,8 +891,8 @@ static int check_work_area(dec_ctx* c) {
     const int cap = o.pro == PRO_MLA_COMBINE ? kCombineOff : kWorkBytes;
     if ((long long)o.Kpad * (o.in_bf16 ? 2 : 4) > cap)
       return fail(c, DEC_ERR_UNSUPPORTED, "input vector of op %zu (%s) exceeds the work area", i, nm);
-    if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.src) || !al(o.gate) || !al(o.up) || o.slot_stride % 4 ||
-        o.gstride % 4 || o.hdim % 4)
+    if (o.n % 4 || o.Kpad % 4 || !al(o.add) || !al(o.add2) || !al(o.routed) || !al(o.src) || !al(o.gate) ||
+        !al(o.up) || o.routed_slot_stride % 4 || o.slot_stride % 4 || o.gstride % 4 || o.hdim % 4)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): vector lengths and offsets must be multiples of 4", i, nm);
     if (o.pro == PRO_MLA_COMBINE && o.nch > kMaxCombine)
       return fail(c, DEC_ERR_UNSUPPORTED, "op %zu (%s): too many split-KV chunks", i, nm);
@@ -993,8 +1014,8 @@ extern "C" int dec_create(const dec_config* cfg, dec_ctx** out) {
       }
     }
   }
-  if ((rc = setup_cursors(c))) return rc;
   if ((rc = upload_ops(c))) return rc;
+  if ((rc = assign_tasks(c))) return rc;
   if ((rc = dalloc(c, &c->d_state, sizeof(StepState)))) return rc;
   if ((rc = dalloc(c, &c->d_gen, sizeof(GenState)))) return rc;
   CK(cudaMemsetAsync(c->d_gen, 0, sizeof(GenState), c->stream));
@@ -1068,7 +1089,6 @@ extern "C" int dec_reset(dec_ctx* c) {
   cudaStreamSynchronize(c->stream);
   (void)cudaGetLastError();
   CK(cudaMemsetAsync(c->d_counters, 0, c->n_counters * 4, c->stream));
-  for (auto& a : c->accs) CK(cudaMemsetAsync(a.first, 0, a.second, c->stream));
   CK(cudaMemsetAsync(c->d_started, 0, 4, c->stream));
   CK(cudaMemsetAsync(c->d_status, 0, sizeof(Status), c->stream));
   CK(cudaMemsetAsync(c->d_gen, 0, sizeof(GenState), c->stream));
@@ -1131,7 +1151,7 @@ static int load_matrix(dec_ctx* c, Mat& m, int expert, const void* data, const f
   uint8_t* dst = m.w + (size_t)expert * m.tile_bytes;
   const long long total16 = (long long)(m.tile_bytes / 16);
   const int grid = (int)std::min<long long>((total16 + 255) / 256, 148 * 16);
-  relayout16<<<std::max(grid, 1), 256, 0, c->stream>>>(src, m.N, m.K, m.wb, m.R, m.nst, m.kcb, total16, dst);
+  relayout16<<<std::max(grid, 1), 256, 0, c->stream>>>(src, m.N, m.K, m.wb, m.R, m.S, m.nst, m.kcb, total16, dst);
   CK(cudaGetLastError());
   if (m.sc_count) CK(cudaMemcpyAsync(m.sc + (size_t)expert * m.sc_count, scales, m.sc_count * 4, cudaMemcpyDefault, c->stream));
   CK(cudaStreamSynchronize(c->stream));
@@ -1154,7 +1174,7 @@ static int load_kvb(dec_ctx* c, int layer, const void* data, const float* scales
     Mat& m = c->mats[{DEC_W_KV_B * 16 + mode, layer}];
     const long long total = (long long)m.tile_bytes;
     const int grid = (int)std::min<long long>((total + 255) / 256, 148 * 16);
-    relayout_kvb<<<std::max(grid, 1), 256, 0, c->stream>>>(src, mode, m.N, m.K, m.wb, m.R, m.nst, m.kcb, total,
+    relayout_kvb<<<std::max(grid, 1), 256, 0, c->stream>>>(src, mode, m.N, m.K, m.wb, m.R, m.S, m.nst, m.kcb, total,
                                                            nope, vh, kvl, m.w);
     CK(cudaGetLastError());
   }
@@ -1313,8 +1333,8 @@ static KParams kparams(dec_ctx* c, int persistent, int op, int tok_in) {
   memset(&P, 0, sizeof P);
   P.ops = c->d_ops;
   P.nops = (int)c->ops.size();
-  P.cursors = c->d_cursors;
-  P.ncur = c->n_cursors;
+  P.tasks = c->d_tasks;
+  P.task_off = c->d_task_off;
   P.counters = c->d_counters;
   P.state = c->d_state;
   P.started = c->d_started;
@@ -1649,9 +1669,8 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     for (size_t i = 0; i < c->ops.size(); ++i) {
       const OpDesc& o = c->ops[i];
       snprintf(line, sizeof line,
-               "%zu %s layer=%d kind=%d tasks=%d K=%d Kpad=%d kcb=%d R=%d acc=%d nst=%d segs=%d dep=%d,%d pdep=%d nch=%d\n",
-               i, c->op_names[i].c_str(), o.layer, o.kind, o.ntasks, o.K, o.Kpad, o.kcb, o.R, o.acc ? 1 : 0, o.nst_total,
-               o.nsegs,
+               "%zu %s layer=%d kind=%d tasks=%d K=%d Kpad=%d kcb=%d R=%d S=%d nst=%d segs=%d dep=%d,%d pdep=%d nch=%d\n",
+               i, c->op_names[i].c_str(), o.layer, o.kind, o.ntasks, o.K, o.Kpad, o.kcb, o.R, o.S, o.nst, o.nsegs,
                o.dep[0], o.dep[1], o.pdep, o.nch);
       s += line;
     }
@@ -1665,8 +1684,8 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
     return DEC_OK;
   }
   if (what == DEC_DUMP_STATUS) {
+    static_assert(sizeof(Status) + sizeof(StepState) == 64, "status dump layout");
     const size_t need = sizeof(Status) + sizeof(StepState);
-    static_assert(sizeof(Status) + sizeof(StepState) == 48, "status dump layout");
     if (out_bytes) *out_bytes = need;
     if (!dst) return DEC_OK;
     if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
@@ -1685,21 +1704,9 @@ extern "C" int dec_debug_dump(dec_ctx* c, int32_t what, void* dst, size_t bytes,
   }
   if (what >= DEC_DUMP_OP && what < DEC_DUMP_OP + (int)c->ops.size()) {
     const OpDesc& o = c->ops[what - DEC_DUMP_OP];
-    if (o.kind == OP_GEMV && o.acc) {  // the last step's accumulator copy, converted to fp32
-      const size_t need = (size_t)o.out_stride * 4;
-      if (out_bytes) *out_bytes = need;
-      if (!dst) return DEC_OK;
-      if (bytes < need) return fail(c, DEC_ERR_INVALID_ARG, "dump needs %zu bytes", need);
-      std::vector<long long> a(o.out_stride);
-      const int par = (c->epoch - 1) & 1;
-      CK(cudaMemcpy(a.data(), o.acc + (size_t)par * o.out_stride, a.size() * 8, cudaMemcpyDeviceToHost));
-      float* f32 = reinterpret_cast<float*>(dst);
-      for (size_t i = 0; i < a.size(); ++i) f32[i] = (float)((double)a[i] * (1.0 / 1099511627776.0));
-      return DEC_OK;
-    }
     std::vector<std::pair<const float*, size_t>> parts;
     if (o.kind == OP_GEMV) {
-      parts.push_back({o.out, (size_t)o.out_stride});
+      parts.push_back({o.out, (size_t)o.S * o.out_stride});
     } else if (o.kind == OP_ATTN || o.kind == OP_MLA) {
       const int heads = o.kind == OP_ATTN ? o.hq : o.H, dim = o.kind == OP_ATTN ? o.hd : o.kvl;
       parts.push_back({o.m_out, (size_t)heads * o.nch});

@@ -8,7 +8,6 @@
 // mechanism the pages describe for TileRT's engine ("Tile A1 + Tile B1 +
 // comm C1", TileRT 是什么 §二 2.2; InferenceX article, "what TileRT is").
 #pragma once
-#include <stddef.h>
 #include <stdint.h>
 
 namespace dec {
@@ -26,7 +25,6 @@ constexpr int kMaxTopK = 16;
 constexpr int kMaxD = 8192;                      // longest normalised vector (d_model, q_lora)
 constexpr int kMlaHeads = 128;                   // MLA attention: heads are the MMA's M dimension (zero-padded)
 constexpr int kMlaBlock = 64;                    // MLA attention: cache positions per block and per task
-constexpr int kPieceStages = 8;                  // GEMV: longest task, in ring stages (longer row tiles are cut along K)
 
 enum WType : int { WT_F32 = 0, WT_BF16 = 1, WT_FP8 = 2 };
 
@@ -64,32 +62,17 @@ DEC_HD constexpr long long mla_q_off(int h, int d) {  // bytes
 enum OpKind : int { OP_GEMV = 0, OP_ATTN = 1, OP_MLA = 2, OP_FINAL = 3 };
 enum Pro : int {
   PRO_NONE = 0,
-  PRO_RESID_NORM = 1,   // h = base + the previous block's output; x = R(rmsnorm(h) * g)
+  PRO_RESID_NORM = 1,   // h = base + partial sums (+ routed experts); x = R(rmsnorm(h) * g)
   PRO_NORM_SUM = 2,     // x = R(rmsnorm(sum of partials) * g)
   PRO_SUM = 3,          // x = R(sum of partials) (optionally per input group)
   PRO_SWIGLU = 4,       // x = R(silu(gate) * up)
   PRO_MLA_COMBINE = 6   // x = R(split-KV combine of one head's latent output)
 };
 
-// Fixed-point accumulators.  Every vector one op hands to another (GEMV outputs,
-// the dense attention's combined output) is held as 64-bit integers in units of
-// 2^-40.  A GEMV whose row tiles are split along K among tasks (and the experts,
-// whose slots all add into one vector) sums its pieces with integer atomics:
-// integer addition is exact and associative, so the sum does not depend on the
-// order in which CTAs finish and the step stays bit-reproducible; a vector written
-// by one task per row is stored plainly.  Readers have one path (two 16-byte loads
-// per four values).  Range +-2^22 (a larger or non-finite value is reported as a
-// numeric error); resolution 2^-40.  Every accumulator has two copies used by
-// alternate steps (parity = epoch & 1): a step adds into its own copy and clears
-// the other one, which the previous step finished with.
-constexpr float kAccScale = 1099511627776.0f;  // 2^40
-constexpr float kAccInv = 1.0f / 1099511627776.0f;
-constexpr float kAccMax = 4194304.0f;          // 2^22
-
-// value(e) = acc[par * stride + off + e] * 2^-40 for the step's parity par (acc null: unused)
+// value(e) = sum_{s < S} ptr[s * stride + off + e]
 struct PSet {
-  const long long* acc;
-  int stride, off;
+  const float* ptr;
+  int S, stride, off;
 };
 
 struct Seg {
@@ -101,40 +84,22 @@ struct Seg {
   int N;              // rows
   int ntiles;         // row tiles of R rows
   int task0;          // first task of this segment within the op
-  int out_off;        // element offset of row 0 in the op's output
+  int out_off;        // element offset of row 0 in every split's output
   int in_group;       // prologue input variant shared by all tasks of the segment (-1: by row group)
-  int zero_acc;       // accumulator ops: this segment's pieces that start at stage 0 clear the other parity
 };
 
-// Tasks are handed out at run time: when a CTA's producer warp reaches an op it takes
-// the op's tasks one at a time from a global cursor (an atomic add) until none is
-// left, streams each task's bytes and passes the task to its consumers through a
-// shared-memory queue.  An SM that streams faster takes more tasks, so an op ends
-// when the last task ends, not when the slowest SM's fixed share does.  An op whose
-// tasks read different input vectors (the routed experts' down projections: one
-// SwiGLU input per slot) has one cursor per input group; a CTA starts at the group
-// its index maps to and moves on to the next group when one runs dry, so most CTAs
-// build one input vector.  Cursors come in two copies used by alternate steps; the
-// final op clears the copy of the next step.
 struct alignas(16) OpDesc {
-  // head (first 32 bytes, read alone by the task hand-out)
   int kind, ntasks, layer;
-  int ngroups, cur_off, trace_base;  // task groups, their first cursor, first trace record
-  const int* gbegin;                 // first task of each group [ngroups + 1] (null: one group of all tasks)
   int dep[2];  // consumer dependencies (op index or -1)
   int pdep;    // producer dependency: router op whose top-k picks the weights of routed segments
-  // ---- GEMV geometry: a unit = R rows x nst consecutive stages of kc columns (a piece of one
-  // row tile); weights are stored [row tile][nst_total stages][R rows][kcb bytes]
-  int wtype, K, Kpad, kcb, kc, cpr, G, rpt, R, nst_total;
+  // ---- GEMV geometry: a task = R rows x (nst stages of kc columns)
+  int wtype, K, Kpad, kcb, kc, cpr, G, rpt, R, S, nst;
   int nsegs;
   Seg seg[kMaxSegs];
-  const int4* pieces;  // per unit: x = segment, y = row tile, z = first stage, w = stages
   int rows_per_group;  // grouped GEMV: input group = row / rows_per_group (0: one input for all rows)
-  int tpt;             // GEMV units per task (0 or 1: one); a task's units share an input group
+  int tpt;             // GEMV units (row tile x split) per task (0 or 1: one); a task's units share a group
   void* qc;            // MLA: absorbed bf16 query in the tensor-core layout (written by absorb_q, read by attention)
-  float* out;          // fp32 outputs [out_stride] (the LM head's logits), or null when acc is set
-  long long* acc;      // fixed-point output [2][out_stride]: stored (one task per row) or added (acc_add)
-  int acc_add;         // the op's tasks split rows along K or add segments into the same rows
+  float* out;          // fp32 partial outputs [S][out_stride]
   int out_stride;
   unsigned long long* best;  // LM head: best packed (value, index) key per task, else null
   // ---- prologue
@@ -145,14 +110,14 @@ struct alignas(16) OpDesc {
   const void* embed;
   int embed_bf16;
   const float* h_base;
-  PSet add;                // added to the base (ptr and acc null = unused); the FFN outputs of an MoE
-                           // layer (routed experts weighted, shared expert) arrive as one accumulator
+  PSet add, add2;          // summed with weight 1 (ptr null = unused)
+  PSet routed;             // routed expert outputs, slot j at off + j * routed_slot_stride
+  int routed_slot_stride;
   int n_experts, top_k;
   int router;              // 1: the router GEMV; its last task turns the logits into the top-k
   unsigned* fin;           // router: tasks finished (cumulative over steps), to find the last one
   int* rt_ids;             // router: top-k expert ids it writes; routed GEMV ops: ids their producer reads
-  float* rt_w;             // router: renormalised top-k weights it writes; RESID_NORM: weights it reads;
-                           // routed GEMV with an accumulator: slot weights applied before the add
+  float* rt_w;             // router: renormalised top-k weights it writes; RESID_NORM: weights it reads
   int* route_dump;         // router: the chosen expert ids are also stored here (debug dump)
   const float* gain;
   float eps;
@@ -183,8 +148,8 @@ struct alignas(16) OpDesc {
   float* m_out;
   float* l_out;
   float* o_out;
-  long long* o_fin;  // dense: combined attention output [2][hq][hd], fixed point (the last chunk task of a
-                    // kv head writes it; `fin` then holds one finished-task counter per kv head)
+  float* o_fin;  // dense: combined attention output [hq][hd] (the last chunk task of a kv head writes it;
+                 // `fin` then holds one finished-task counter per kv head)
   int np;  // positions per ring stage
   // ---- final op
   const unsigned long long* fin_best;
@@ -192,7 +157,6 @@ struct alignas(16) OpDesc {
   int vocab;
   float* logits;  // LM head output (the final op reads nothing from it; kept for dumps)
 };
-static_assert(offsetof(OpDesc, gbegin) == 24, "the task hand-out reads the descriptor head as int4 + pointer");
 
 struct StepState {
   int epoch;  // 1-based step counter since the last reset (dependency counter targets)
@@ -215,13 +179,15 @@ struct GenState {
 struct Status {
   int code;  // 0 ok, 1 a bounded wait timed out, 2 a non-finite router or LM-head logit
   int cta, op, task;
+  unsigned long long final_key;  // the last final op's winning (order-preserving logit bits, ~index) key
+  unsigned long long pad;
 };
 
 struct KParams {
   const OpDesc* ops;
   int nops;
-  unsigned* cursors;     // task cursors [2][ncur] (copy epoch & 1 is this step's)
-  int ncur;
+  const int2* tasks;     // (op, task) pairs of all CTAs
+  const int* task_off;   // CTA b runs tasks[task_off[b] .. task_off[b + 1])
   unsigned* counters;    // one per op, cumulative over steps
   StepState* state;
   unsigned* started;     // CTAs that have read the step state (cumulative)

@@ -30,7 +30,6 @@
 namespace dec {
 
 constexpr int kMail = 16;  // mailbox slots between consumers and the signaller
-constexpr int kTQ = 16;    // task queue slots between the producer and the consumers
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kSignalWarp = kConsumerWarps + 1;
 constexpr int kOdBytes = (int)((sizeof(OpDesc) + 15) / 16 * 16);
@@ -52,15 +51,8 @@ struct Misc {
   int issued;            // ring stages issued (producer lane 0)
   int prod_route_op;     // router op whose top-k is in prod_idx
   int prod_idx[kMaxTopK];
+  float cons_w[kMaxTopK];
   int mail_op[kMail], mail_task[kMail];
-  uint64_t tq_full[kTQ];   // producer -> consumers: task in queue slot (op, task, unit geometry)
-  uint64_t tq_empty[kTQ];  // consumers -> producer: queue slot read
-  int tq_op[kTQ], tq_t[kTQ];
-  int4 tq_geo[kTQ];
-  int4 tq_st[kTQ];         // the task's step: epoch, position, token, 0
-  int cur_op, cur_t;       // the task the consumers run (copied out of the queue by thread 0)
-  int4 cur_geo;
-  int new_step;            // the task is the consumers' first of a new step
   unsigned long long mail_t[kMail][4];  // trace: task start, input vector ready, first stage available, compute done
   unsigned long long tr_pro;            // trace: when the current task's input vector was ready
   unsigned long long tr_data;           // trace: when the current task's first stage was available
@@ -116,15 +108,18 @@ __device__ __noinline__ void report_nonfinite(const KParams& P, int op, int task
   }
 }
 
+// true unless v is an infinity or a NaN (all exponent bits set), tested on the bits
+__device__ __forceinline__ bool finite_bits(float v) { return (__float_as_uint(v) & 0x7F800000u) != 0x7F800000u; }
+
 // Spin until ready(); false if this CTA gave up (deadline passed or the CTA's
 // abort flag set).  Waits on another CTA (cross_cta) also watch the global status
 // word, so that a failure anywhere stops them; waits inside the CTA only read
 // the CTA's own flag (many threads spin on those: they must not load global
 // memory while they wait).
-// The spin loop is out of line (one copy per kind of wait); the first test is inline.
 template <class F>
-__device__ __noinline__ bool bounded_wait_slow(F ready, const KParams& P, volatile int* abort, int op, int task,
-                                               bool cross_cta) {
+__device__ __forceinline__ bool bounded_wait(F ready, const KParams& P, volatile int* abort, int op, int task,
+                                             bool cross_cta) {
+  if (ready()) return true;
   const uint64_t t0 = globaltimer();
   for (unsigned it = 1;; ++it) {
     if (ready()) return true;
@@ -142,13 +137,6 @@ __device__ __noinline__ bool bounded_wait_slow(F ready, const KParams& P, volati
     }
     if (cross_cta) __nanosleep(64);
   }
-}
-
-template <class F>
-__device__ __forceinline__ bool bounded_wait(F ready, const KParams& P, volatile int* abort, int op, int task,
-                                             bool cross_cta) {
-  if (ready()) return true;
-  return bounded_wait_slow(ready, P, abort, op, task, cross_cta);
 }
 
 __device__ __forceinline__ bool wait_counter(const KParams& P, int dop, unsigned epoch, volatile int* abort,
@@ -190,17 +178,11 @@ __device__ __forceinline__ float consumer_sum(float v, Misc* m) {
 }
 
 // ---------------------------------------------------------------- helpers
-__device__ __forceinline__ float acc_value(long long a) { return __ll2float_rn(a) * kAccInv; }
-
-// true unless v is an infinity or a NaN (all exponent bits set), tested on the bits
-__device__ __forceinline__ bool finite_bits(float v) { return (__float_as_uint(v) & 0x7F800000u) != 0x7F800000u; }
-
-__device__ __forceinline__ float pset(const PSet& p, int e, int par) {
-  return acc_value(__ldcg(p.acc + (size_t)par * p.stride + p.off + e));
+__device__ __forceinline__ float pset(const PSet& p, int e) {
+  float v = 0.f;
+  for (int s = 0; s < p.S; ++s) v += ldcg(p.ptr + (size_t)s * p.stride + p.off + e);
+  return v;
 }
-
-// fixed-point value of v for a stored accumulator element (range checked by the caller)
-__device__ __forceinline__ long long acc_fixed(float v) { return __float2ll_rn(v * kAccScale); }
 
 __device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ void add4(float4& a, const float4 b) {
@@ -216,11 +198,12 @@ __device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
   a.w = fmaf(w, b.w, a.w);
 }
 
-// 4 consecutive elements (e multiple of 4): two 16-byte loads.
-__device__ __forceinline__ float4 pset4(const PSet& p, int e, int par) {
-  const longlong2* a = reinterpret_cast<const longlong2*>(p.acc + (size_t)par * p.stride + p.off + e);
-  const longlong2 u = __ldcg(a), w = __ldcg(a + 1);
-  return make_float4(acc_value(u.x), acc_value(u.y), acc_value(w.x), acc_value(w.y));
+// Sum over splits of 4 consecutive elements (e multiple of 4, offsets 16-byte aligned).
+__device__ __forceinline__ float4 pset4(const PSet& p, int e) {
+  const float* b = p.ptr + p.off + e;
+  float4 v = ldcg4(b);  // first split unconditionally, so callers' loads can be issued together
+  for (int s = 1; s < p.S; ++s) add4(v, ldcg4(b + (size_t)s * p.stride));
+  return v;
 }
 
 __device__ __forceinline__ float rnd(float v, int bf16) { return bf16 ? bf16_round(v) : v; }
@@ -249,20 +232,35 @@ __device__ __forceinline__ void store_x4(uint8_t* work, int in_bf16, int e, floa
 // ties to the lower expert id, weights renormalised over the chosen k:
 // w_j = exp(r_j - r_max) / sum_i exp(r_i - r_max).  Returns false (every lane) if
 // any logit is NaN or infinite; the ids and weights are then still written.
-__device__ __forceinline__ bool warp_route(const PSet& logits, int E, int k, int par, int* idx_out, float* w_out) {
+__device__ __forceinline__ bool warp_route(const PSet& logits, int E, int k, int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
   float v[8];
   int taken = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = e < E ? pset(logits, e, par) : 0.f;  // 8 independent loads per lane
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  // sum the split-K partials, 4 splits x 8 logits = 32 independent loads per batch
+  const float* base = logits.ptr + logits.off;
+  for (int s0 = 0; s0 < logits.S; s0 += 4) {
+    float u[4][8];
+#pragma unroll
+    for (int ds = 0; ds < 4; ++ds)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        u[ds][i] = (s0 + ds < logits.S && e < E) ? ldcg(base + (size_t)(s0 + ds) * logits.stride + e) : 0.f;
+      }
+#pragma unroll
+    for (int ds = 0; ds < 4; ++ds)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += u[ds][i];
   }
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    if (lane + 32 * i >= E) v[i] = -INFINITY;
-    else bad |= !finite_bits(v[i]);
+    if (lane + 32 * i >= E)
+      v[i] = -INFINITY;
+    else
+      bad |= !finite_bits(v[i]);
   }
   bad = __any_sync(0xffffffffu, bad);
   float top[kMaxTopK];
@@ -342,11 +340,14 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
   uint8_t* x = S.work;
   const int n = od.n;
   const int bf = od.in_bf16;
-  const int par = m->st.epoch & 1;
   switch (od.pro) {
     case PRO_RESID_NORM:
     case PRO_NORM_SUM: {
       const bool resid = od.pro == PRO_RESID_NORM;
+      if (resid && od.routed.ptr) {
+        if (tid < od.top_k) m->cons_w[tid] = __ldcg(od.rt_w + tid);  // written by the router's last task
+        named_bar_sync(1, kConsumers);
+      }
       float4 v[kMaxQ];
       // The gains (often read from HBM) are copied asynchronously into the work area
       // behind the input vector, so their latency overlaps the base and source loads;
@@ -358,35 +359,66 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         for (int e = 4 * tid; e < n; e += 4 * kConsumers) cp_async16(gs + e, od.gain + e);
         cp_async_commit();
       }
-      // h = base + add (one vector: the previous op's output, fp32 or accumulator), all
-      // loads of a thread issued before any is used
-      float4 u[kMaxQ];
+      // base
 #pragma unroll
       for (int i = 0; i < kMaxQ; ++i) {
         const int e = 4 * (tid + i * kConsumers);
         v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        u[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (e < n) {
           if (!resid) {
-            v[i] = pset4(od.src, e, par);
-          } else {
-            if (od.base_embed) {
-              const size_t row = (size_t)m->st.tok * n;
-              if (od.embed_bf16) {
-                const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(od.embed) + row + e));
-                v[i] = make_float4(bf16lo(w2.x), bf16hi(w2.x), bf16lo(w2.y), bf16hi(w2.y));
-              } else {
-                v[i] = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(od.embed) + row + e));
-              }
+            v[i] = pset4(od.src, e);
+          } else if (od.base_embed) {
+            const size_t row = (size_t)m->st.tok * n;
+            if (od.embed_bf16) {
+              const uint2 u = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(od.embed) + row + e));
+              v[i] = make_float4(bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y));
             } else {
-              v[i] = ldcg4(od.h_base + e);
+              v[i] = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(od.embed) + row + e));
             }
-            if (od.add.acc) u[i] = pset4(od.add, e, par);
+          } else {
+            v[i] = ldcg4(od.h_base + e);
           }
         }
       }
+      if (resid) {
+        // Added sources: every split of `add` and `add2` (weight 1) and of each routed
+        // expert slot j (weight w_j).  kSrcBatch sources are loaded per batch so
+        // that each thread has up to kSrcBatch * kMaxQ 16-byte loads in flight.
+        const int na = od.add.ptr ? od.add.S : 0, nb = od.add2.ptr ? od.add2.S : 0;
+        const int nr = od.routed.ptr ? od.top_k * od.routed.S : 0;
+        const int nsrc = na + nb + nr;
+        auto src = [&](int k, float& wk) -> const float* {
+          wk = 1.f;
+          if (k < na) return od.add.ptr + od.add.off + (size_t)k * od.add.stride;
+          k -= na;
+          if (k < nb) return od.add2.ptr + od.add2.off + (size_t)k * od.add2.stride;
+          k -= nb;
+          const int j = k / od.routed.S, s = k % od.routed.S;
+          wk = m->cons_w[j];
+          return od.routed.ptr + od.routed.off + (size_t)j * od.routed_slot_stride + (size_t)s * od.routed.stride;
+        };
+        for (int k0 = 0; k0 < nsrc; k0 += kSrcBatch) {
+          float w3[kSrcBatch];
+          const float* p3[kSrcBatch];
+          float4 u[kSrcBatch][kMaxQ];
 #pragma unroll
-      for (int i = 0; i < kMaxQ; ++i) add4(v[i], u[i]);
+          for (int b = 0; b < kSrcBatch; ++b) {
+            p3[b] = k0 + b < nsrc ? src(k0 + b, w3[b]) : nullptr;
+            if (!p3[b]) w3[b] = 0.f;
+          }
+#pragma unroll
+          for (int b = 0; b < kSrcBatch; ++b)
+#pragma unroll
+            for (int i = 0; i < kMaxQ; ++i) {
+              const int e = 4 * (tid + i * kConsumers);
+              u[b][i] = (p3[b] && e < n) ? ldcg4(p3[b] + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+          for (int b = 0; b < kSrcBatch; ++b)
+#pragma unroll
+            for (int i = 0; i < kMaxQ; ++i) fma4(v[i], w3[b], u[b][i]);  // w = 1: exact add
+        }
+      }
       float ss = 0.f;
 #pragma unroll
       for (int i = 0; i < kMaxQ; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
@@ -418,7 +450,7 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int e = e0 + u * 4 * kConsumers;
-          if (e < n) v[u] = pset4(p, e, par);
+          if (e < n) v[u] = pset4(p, e);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -438,8 +470,8 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
         for (int u = 0; u < 4; ++u) {
           const int e = e0 + u * 4 * kConsumers;
           if (e < n) {
-            gv[u] = pset4(gp, e, par);
-            uv[u] = pset4(up, e, par);
+            gv[u] = pset4(gp, e);
+            uv[u] = pset4(up, e);
           }
         }
 #pragma unroll
@@ -497,63 +529,21 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
 }
 
 // ------------------------------------------------------------ GEMV tasks
-// A unit: segment si, row tile rt, stages [st0, st0 + nst) of the tile's K range.
 struct TaskGeo {
-  int si, rt, st0, nst, group;
+  int si, rt, s, group;
 };
 
-// Ops with a piece table (row tiles split along K, accumulator output) read the unit
-// from it; the others run whole row tiles, numbered segment by segment.
-__device__ __forceinline__ TaskGeo gemv_geo(const OpDesc& od, int u, int4 pc) {
+__device__ __forceinline__ TaskGeo gemv_geo(const OpDesc& od, int t) {
   TaskGeo g;
-  if (od.pieces) {  // pc: the unit's entry of the piece table (one unit per task)
-    g.si = pc.x;
-    g.rt = pc.y;
-    g.st0 = pc.z;
-    g.nst = pc.w;
-  } else {
-    int si = 0;
-    while (si + 1 < od.nsegs && u >= od.seg[si + 1].task0) ++si;
-    g.si = si;
-    g.rt = u - od.seg[si].task0;
-    g.st0 = 0;
-    g.nst = od.nst_total;
-  }
-  const Seg& sg = od.seg[g.si];
+  int si = 0;
+  while (si + 1 < od.nsegs && t >= od.seg[si + 1].task0) ++si;
+  const Seg& sg = od.seg[si];
+  const int local = t - sg.task0;
+  g.si = si;
+  g.rt = local / od.S;
+  g.s = local % od.S;
   g.group = sg.in_group >= 0 ? sg.in_group : (od.rows_per_group ? (g.rt * od.R) / od.rows_per_group : 0);
   return g;
-}
-
-// One GEMV output row (out of line: the epilogue calls it once per row a thread holds).
-// fp32 (logits), stored fixed point, or added fixed point (weighted by the routed slot's
-// router weight; the pieces that start a tile's K range also clear the other parity);
-// absorb_q's rows also go to the tensor-core query in bf16.
-__device__ __noinline__ void put_row(const KParams& P, const OpDesc& od, int out_off, long long* acc_out,
-                                     long long* acc_clr, float wslot, int row, float y, int op, int t);
-
-// Adds v into a fixed-point accumulator element (one red.global.add.u64).
-__device__ __forceinline__ void acc_add(const KParams& P, long long* a, float v, int op, int t) {
-  if (!(fabsf(v) < kAccMax)) {  // NaN, infinite or out of the accumulator's range
-    report_nonfinite(P, op, t);
-    return;
-  }
-  atomicAdd(reinterpret_cast<unsigned long long*>(a), (unsigned long long)__float2ll_rn(v * kAccScale));
-}
-
-__device__ __noinline__ void put_row(const KParams& P, const OpDesc& od, int out_off, long long* acc_out,
-                                     long long* acc_clr, float wslot, int row, float y, int op, int t) {
-  if (!acc_out) {
-    od.out[out_off + row] = y;
-  } else if (!od.acc_add) {
-    if (!(fabsf(y) < kAccMax)) report_nonfinite(P, op, t);
-    acc_out[row] = acc_fixed(y);
-  } else {
-    acc_add(P, acc_out + row, wslot * y, op, t);
-    if (acc_clr) acc_clr[row] = 0;
-  }
-  if (od.qc)
-    reinterpret_cast<__nv_bfloat16*>(od.qc)[mla_q_off(row / od.rows_per_group, row % od.rows_per_group) / 2] =
-        __float2bfloat16_rn(y);
 }
 
 __device__ __forceinline__ void wait_full(const KParams& P, const Smem& S, uint32_t g, int op, int task) {
@@ -565,8 +555,14 @@ __device__ __forceinline__ void release_stage(const Smem& S, uint32_t g) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(&S.m->empty[g % kStages]);
 }
 
+// Order-preserving key of (logit, index): larger logit wins, then the smaller index.
+// The bits are taken through an opaque move so that the sign-bit or/xor below stays
+// integer work: written on a plain bitcast, the compiler may turn it into float
+// negate/absolute-value, whose result for a NaN input is an unspecified NaN, and a NaN
+// logit must keep its all-ones key for the final op to see it.
 __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
-  uint32_t u = __float_as_uint(v);
+  uint32_t u;
+  asm("mov.b32 %0, %1;" : "=r"(u) : "f"(v));
   u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
   return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (uint32_t)idx);
 }
@@ -654,7 +650,7 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
   Misc* m = S.m;
   const int tid = threadIdx.x;
   const int c = tid % CPR, rg = tid / CPR;
-  const int nst = geo.nst;
+  const int nst = od.nst;
   float acc[RPT];
 #pragma unroll
   for (int i = 0; i < RPT; ++i) acc[i] = 0.f;
@@ -668,7 +664,7 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
     wait_full(P, S, g, op, t);  // on failure the task runs to its end on stale data; the caller stops after it
     if (P.trace && st == 0 && tid == 0) m->tr_data = globaltimer();
     const uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
-    const int k0 = (geo.st0 + st) * KC;
+    const int k0 = (geo.s * nst + st) * KC;
     float scale = 1.f;
     if constexpr (WT == WT_FP8) {
       if (st == 0 && sg.slot >= 0) {  // the producer wrote the expert id before this stage's copy
@@ -687,22 +683,19 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
   for (int o = SPAN >> 1; o > 0; o >>= 1)
 #pragma unroll
     for (int i = 0; i < RPT; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-  const int par = m->st.epoch & 1;
-  long long* acc_out = nullptr;
-  long long* acc_clr = nullptr;
-  float wslot = 1.f;
-  if (od.acc) {
-    acc_out = od.acc + (size_t)par * od.out_stride + sg.out_off;
-    if (od.acc_add && sg.zero_acc && geo.st0 == 0) acc_clr = od.acc + (size_t)(par ^ 1) * od.out_stride + sg.out_off;
-    if (sg.slot >= 0 && od.rt_w) wslot = __ldcg(od.rt_w + sg.slot);  // the op depends on the router
-  }
   if (PARTS == 1 && !od.best) {
     // a row's chunks all live in one warp: its first lane holds the row sum, no CTA barrier needed
     if ((lane & (SPAN - 1)) == 0) {
+      float* out = od.out + (size_t)geo.s * od.out_stride + sg.out_off;
 #pragma unroll
       for (int i = 0; i < RPT; ++i) {
         const int row = geo.rt * R + rg + G * i;
-        if (row < sg.N) put_row(P, od, sg.out_off, acc_out, acc_clr, wslot, row, acc[i], op, t);
+        if (row < sg.N) {
+          out[row] = acc[i];
+          if (od.qc)
+            reinterpret_cast<__nv_bfloat16*>(od.qc)[mla_q_off(row / od.rows_per_group, row % od.rows_per_group) / 2] =
+                __float2bfloat16_rn(acc[i]);
+        }
       }
     }
     return;
@@ -721,7 +714,10 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
     for (int p = 0; p < PARTS; ++p) y += m->red[(i * G + rg2) * PARTS + p];
     const int row = geo.rt * R + tid;
     if (row < sg.N) {
-      put_row(P, od, sg.out_off, acc_out, acc_clr, wslot, row, y, op, t);
+      od.out[(size_t)geo.s * od.out_stride + sg.out_off + row] = y;
+      if (od.qc)
+        reinterpret_cast<__nv_bfloat16*>(od.qc)[mla_q_off(row / od.rows_per_group, row % od.rows_per_group) / 2] =
+            __float2bfloat16_rn(y);
       if (od.best) key = argmax_key(y, sg.out_off + row);
     }
   }
@@ -746,11 +742,11 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
 // (all consumer threads; absorb_q's extra last task, before attention reads the block).
 __device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
   Misc* m = S.m;
-  const int tid = threadIdx.x, pos = m->st.pos, par = m->st.epoch & 1;
+  const int tid = threadIdx.x, pos = m->st.pos;
   const int kvl = od.rows_per_group, rd = od.rdim, rowe = kvl + rd;
   __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(S.work + kCombineOff);  // [rowe]
   float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (4 * tid < kvl) v = pset4(od.ckv, 4 * tid, par);  // 16-byte loads (or accumulator pairs)
+  if (4 * tid < kvl) v = pset4(od.ckv, 4 * tid);  // 16-byte loads of the split partials
   const float tot = consumer_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w, m);
   const float inv = 1.0f / sqrtf(tot / (float)kvl + od.eps);
   if (4 * tid < kvl) {
@@ -761,7 +757,7 @@ __device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
   const int rq = tid - kvl / 4;  // RoPE: 4 pairs (j, j + rd/2) per thread
   if (rq >= 0 && 4 * rq < rd / 2) {
     const int j = 4 * rq;
-    const float4 a = pset4(od.ckv, kvl + j, par), b = pset4(od.ckv, kvl + j + rd / 2, par);
+    const float4 a = pset4(od.ckv, kvl + j), b = pset4(od.ckv, kvl + j + rd / 2);
     const float4 cs = __ldg(reinterpret_cast<const float4*>(od.rope_cos + (size_t)pos * (rd / 2) + j));
     const float4 sn = __ldg(reinterpret_cast<const float4*>(od.rope_sin + (size_t)pos * (rd / 2) + j));
     __nv_bfloat162* lo = reinterpret_cast<__nv_bfloat162*>(row + kvl + j);
@@ -780,17 +776,21 @@ __device__ __forceinline__ void mla_new_row(const OpDesc& od, const Smem& S) {
 template <int WT>
 __device__ __forceinline__ void gemv_unit(const KParams& P, const OpDesc& od, int op, int u, const Smem& S,
                                           uint32_t& g, const TaskGeo& geo) {
-  switch (od.kcb) {  // the stage widths the planner picks (gemv_geometry)
+  switch (od.kcb) {
+    case 4096: gemv_task<WT, 4096>(P, od, op, u, S, g, geo); break;
+    case 2048: gemv_task<WT, 2048>(P, od, op, u, S, g, geo); break;
+    case 1024: gemv_task<WT, 1024>(P, od, op, u, S, g, geo); break;
     case 512: gemv_task<WT, 512>(P, od, op, u, S, g, geo); break;
     case 256: gemv_task<WT, 256>(P, od, op, u, S, g, geo); break;
     case 128: gemv_task<WT, 128>(P, od, op, u, S, g, geo); break;
-    default: gemv_task<WT, 64>(P, od, op, u, S, g, geo); break;
+    case 64: gemv_task<WT, 64>(P, od, op, u, S, g, geo); break;
+    default: gemv_task<WT, 32>(P, od, op, u, S, g, geo); break;
   }
 }
 
 template <int WT>
 __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od, int op, int t, const Smem& S,
-                                             uint32_t& g, int4 pc) {
+                                             uint32_t& g) {
   Misc* m = S.m;
   if (od.qc && t == od.ntasks - 1) {  // absorb_q's extra task: the step's latent cache row
     mla_new_row(od, S);
@@ -800,7 +800,7 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
   const int tpt = od.tpt > 1 ? od.tpt : 1;
   for (int i = 0; i < tpt; ++i) {  // a task's units (row tiles) share the input group
   const int u = t * tpt + i;
-  const TaskGeo geo = gemv_geo(od, u, pc);
+  const TaskGeo geo = gemv_geo(od, u);
   if (m->x_op != op || m->x_group != geo.group) {
     prologue(od, geo.group, u, S);
     if (threadIdx.x == 0) {
@@ -822,7 +822,7 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
     named_bar_sync(1, kConsumers);
     if (m->last_task && threadIdx.x < 32) {
       __threadfence();
-      if (!warp_route(PSet{od.acc, od.out_stride, 0}, od.n_experts, od.top_k, m->st.epoch & 1, od.rt_ids, od.rt_w) &&
+      if (!warp_route(PSet{od.out, od.S, od.out_stride, 0}, od.n_experts, od.top_k, od.rt_ids, od.rt_w) &&
           threadIdx.x == 0)
         report_nonfinite(P, op, t);
       if (od.route_dump && threadIdx.x < od.top_k) od.route_dump[threadIdx.x] = __ldcg(od.rt_ids + threadIdx.x);
@@ -831,13 +831,12 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
   if (od.qc) {
     // absorb_q also feeds the tensor-core MLA attention: gemv_task stored q_lat
     // rows in bf16; the first tile of head h adds its RoPE'd q_pe (bf16).
-    if (geo.st0 == 0 && (geo.rt * od.R) % od.rows_per_group == 0) {
+    if (geo.s == 0 && (geo.rt * od.R) % od.rows_per_group == 0) {
       const int h = geo.rt * od.R / od.rows_per_group, rd = od.rdim, kvl = od.rows_per_group;
-      const int pos = m->st.pos, pos_par = m->st.epoch & 1;
+      const int pos = m->st.pos;
       __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(od.qc);
       for (int j = threadIdx.x; j < rd / 2; j += kConsumers) {
-        const float a = pset(od.src, h * od.gstride + od.nope + j, pos_par),
-                    b = pset(od.src, h * od.gstride + od.nope + j + rd / 2, pos_par);
+        const float a = pset(od.src, h * od.gstride + od.nope + j), b = pset(od.src, h * od.gstride + od.nope + j + rd / 2);
         const float cs = od.rope_cos[(size_t)pos * (rd / 2) + j], sn = od.rope_sin[(size_t)pos * (rd / 2) + j];
         q[mla_q_off(h, kvl + j) / 2] = __float2bfloat16_rn(a * cs - b * sn);
         q[mla_q_off(h, kvl + j + rd / 2) / 2] = __float2bfloat16_rn(a * sn + b * cs);
@@ -946,7 +945,7 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
   const int set = warp / WPS, wi = warp % WPS;
   const int nch = od.nch, np = od.np;
   const int kvh = t / nch, c = t % nch;
-  const int pos = m->st.pos, par = m->st.epoch & 1;
+  const int pos = m->st.pos;
   const ChunkB b = chunk_bounds(c, nch, pos);
   const int hd = od.hd, gs = od.gs, cbf = od.cache_bf16, cb = cbf ? 2 : 4;
   const int rowb = hd * cb;
@@ -960,7 +959,7 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
   for (int e = tid; e < gs * half; e += kConsumers) {
     const int i = e / half, j = e % half;
     const int qh = kvh * gs + i;
-    const float a = pset(od.qkv, qh * hd + j, par), bq = pset(od.qkv, qh * hd + j + half, par);
+    const float a = pset(od.qkv, qh * hd + j), bq = pset(od.qkv, qh * hd + j + half);
     q_s[i * hd + j] = rnd(a * cosr[j] - bq * sinr[j], cbf);
     q_s[i * hd + j + half] = rnd(a * sinr[j] + bq * cosr[j], cbf);
   }
@@ -968,7 +967,7 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
     const int koff = od.hq * hd + kvh * hd, voff = (od.hq + od.hkv) * hd + kvh * hd;
     const size_t crow = ((size_t)kvh * od.max_seq + pos) * hd;
     for (int j = tid; j < half; j += kConsumers) {
-      const float a = pset(od.qkv, koff + j, par), bk = pset(od.qkv, koff + j + half, par);
+      const float a = pset(od.qkv, koff + j), bk = pset(od.qkv, koff + j + half);
       const float k0 = rnd(a * cosr[j] - bk * sinr[j], cbf);
       const float k1 = rnd(a * sinr[j] + bk * cosr[j], cbf);
       if (cbf) {
@@ -984,7 +983,7 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
       }
     }
     for (int j = tid; j < hd; j += kConsumers) {
-      const float v = rnd(pset(od.qkv, voff + j, par), cbf);
+      const float v = rnd(pset(od.qkv, voff + j), cbf);
       if (cbf) {
         reinterpret_cast<__nv_bfloat16*>(new_s + rowb)[j] = __float2bfloat16_rn(v);
         reinterpret_cast<__nv_bfloat16*>(od.vcache)[crow + j] = __float2bfloat16_rn(v);
@@ -1141,7 +1140,7 @@ __device__ __forceinline__ void attn_task(const KParams& P, const OpDesc& od, in
         for (int u = 0; u < 8; ++u)
           if (c0 + u < nch) acc = fmaf(wt[h * nch + c0 + u], a[u], acc);
       }
-      od.o_fin[(size_t)(m->st.epoch & 1) * od.hq * hd + (size_t)qh * hd + d] = acc_fixed(acc);
+      od.o_fin[(size_t)qh * hd + d] = acc;
     }
   }
 }
@@ -1344,10 +1343,6 @@ __device__ __forceinline__ void final_consume(const KParams& P, const OpDesc& od
     key = ok > key ? ok : key;
   }
   if (lane == 0) m->redk[warp] = key;
-  // the next step takes its tasks from the other copy of the cursors: clear it (this
-  // step's tasks have all been handed out, or this op would not run)
-  unsigned* nxt = P.cursors + (size_t)((m->st.epoch + 1) & 1) * P.ncur;
-  for (int i = tid; i < P.ncur; i += kConsumers) nxt[i] = 0u;
   named_bar_sync(1, kConsumers);
   if (tid == 0) {
     unsigned long long b = 0ull;
@@ -1371,6 +1366,7 @@ __device__ __forceinline__ void final_consume(const KParams& P, const OpDesc& od
     ns.tok = next;
     ns.last = next;
     ns.stop = 0;
+    ns.pad[0] = ns.pad[1] = ns.pad[2] = 0;
     if (P.gen && __ldcg(&P.gen->active)) {  // generation: the token goes to the host as soon as it is known
       const int s = m->st.epoch - __ldcg(&P.gen->epoch0);
       reinterpret_cast<volatile int*>(P.tok_ring)[s] = next;
@@ -1380,25 +1376,61 @@ __device__ __forceinline__ void final_consume(const KParams& P, const OpDesc& od
         ns.stop = 1;
     }
     *P.state = ns;
+    P.status->final_key = b;  // the winning packed key, for dumps
     if (bad) report_nonfinite(P, op, t);  // after the state: a stopped step still advances consistently
   }
 }
 
+// ------------------------------------------------------------ task lists
+// Walks this CTA's (op, task) list; the entry after the current one is loaded a
+// task ahead so the list read never sits on the critical path.
+struct TaskIter {
+  const int2* list;
+  int i, end, op, stride, persistent;
+  int2 nxt;
+  __device__ void init(const KParams& p) {
+    persistent = p.persistent;
+    if (persistent) {
+      list = p.tasks;
+      i = p.task_off[blockIdx.x];
+      end = p.task_off[blockIdx.x + 1];
+      stride = 1;
+      if (i < end) nxt = __ldg(list + i);
+    } else {
+      list = nullptr;
+      op = p.op_only;
+      i = blockIdx.x;
+      end = __ldg(&p.ops[op].ntasks);
+      stride = gridDim.x;
+    }
+  }
+  __device__ bool next(int& o, int& t) {
+    if (i >= end) return false;
+    if (persistent) {
+      o = nxt.x;
+      t = nxt.y;
+      if (i + 1 < end) nxt = __ldg(list + i + 1);
+    } else {
+      o = op;
+      t = i;
+    }
+    i += stride;
+    return true;
+  }
+};
+
 // --------------------------------------------------------------- producer
-// Walks the ops in order (all of them, or the one op of a per-op launch).  For each op
-// it takes tasks from the op's cursors until they run dry: it hands each task to the
-// consumers through the task queue, then streams the task's stages into the ring.
 __device__ void producer_loop(const KParams& P, const Smem& S) {
   Misc* m = S.m;
   const int lane = threadIdx.x & 31;
   const uint64_t pol_w = policy_evict_first();  // weights: streamed once per step
   const uint64_t pol_kv = policy_evict_last();  // caches: re-read every step
-  uint32_t g = 0, qn = 0;  // ring stages issued, tasks queued
-  int op = -1, t = -1;
-  int pos = m->st.pos;
-  unsigned epoch = (unsigned)m->st.epoch;
-  int4 stv = make_int4((int)epoch, pos, m->st.tok, 0);  // the step every queued task carries
-  unsigned* cursors = P.cursors + (size_t)(epoch & 1) * P.ncur;
+  uint32_t g = 0;
+  TaskIter it;
+  it.init(P);
+  int op, t, cur = -1;
+  const int pos0 = m->st.pos;
+  const unsigned epoch0 = (unsigned)m->st.epoch;
   const OpDesc& od = *S.pod;
   unsigned long long* tr_first = nullptr;  // trace: where the current task's first issue time goes (lane 0)
   auto issue = [&](const void* src, uint32_t bytes, const void* src2, uint32_t bytes2, uint32_t off2,
@@ -1423,95 +1455,51 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
     ++g;
     return true;
   };
-  // Hands (op, t, geometry) to the consumers; op < 0 ends their loop.
-  auto push = [&](int pop, int pt, int4 geo) -> bool {
-    const int slot = qn % kTQ;
-    int ready = 1;
-    if (lane == 0) {
-      ready = mbar_wait(&m->tq_empty[slot], ((qn / kTQ) & 1) ^ 1, P, &m->abort, pop, pt) ? 1 : 0;
-      if (ready) {
-        m->tq_op[slot] = pop;
-        m->tq_t[slot] = pt;
-        m->tq_geo[slot] = geo;
-        m->tq_st[slot] = stv;
-        mbar_arrive(&m->tq_full[slot]);
-      }
-    }
-    ++qn;
-    return __shfl_sync(0xffffffffu, ready, 0) != 0;
-  };
   bool ok = true;
-  int copied = -1;  // op whose descriptor is in shared memory
-  const int op0 = P.persistent ? 0 : P.op_only, op1 = P.persistent ? P.nops : P.op_only + 1;
-  for (int s = 0; s < P.n_steps && ok; ++s) {
-  if (s > 0) {
+  int pos = pos0;
+  unsigned epoch = epoch0;
+  for (int step = 0; step < P.n_steps && ok; ++step) {
+  if (step > 0) {
     // A launch of several steps: the previous step's final op (the last op) wrote this
-    // step's state; take it once that op is published, and stop if it asked to.
-    int r = 0;
+    // step's state; take it once that op is published, and end if it asked to.
+    int r = 0, npos = 0, nep = 0, stop = 0;
     if (lane == 0) {
       r = wait_counter(P, P.nops - 1, epoch, &m->abort, P.nops - 1, 0) ? 1 : 0;
       if (r) {
-        const StepState* gs = P.state;
-        stv = make_int4(__ldcg(&gs->epoch), __ldcg(&gs->pos), __ldcg(&gs->tok), __ldcg(&gs->stop));
-        atomicAdd(P.started, 1u);  // this CTA has read the step's state
+        npos = __ldcg(&P.state->pos);
+        nep = __ldcg(&P.state->epoch);
+        stop = __ldcg(&P.state->stop);
         m->prod_route_op = -1;
         m->prod_dep_op = -1;
       }
     }
-    if (!__shfl_sync(0xffffffffu, r, 0)) {
-      ok = false;
-      break;
-    }
-    stv = make_int4(__shfl_sync(0xffffffffu, stv.x, 0), __shfl_sync(0xffffffffu, stv.y, 0),
-                    __shfl_sync(0xffffffffu, stv.z, 0), __shfl_sync(0xffffffffu, stv.w, 0));
+    if (!__shfl_sync(0xffffffffu, r, 0) || __shfl_sync(0xffffffffu, stop, 0)) break;
+    pos = __shfl_sync(0xffffffffu, npos, 0);
+    epoch = (unsigned)__shfl_sync(0xffffffffu, nep, 0);
     __syncwarp();
-    if (stv.w) break;
-    epoch = (unsigned)stv.x;
-    pos = stv.y;
-    stv.w = 0;
-    cursors = P.cursors + (size_t)(epoch & 1) * P.ncur;
-    copied = -1;
+    it.init(P);
   }
-  for (int oi = op0; oi < op1 && ok; ++oi) {
-    op = oi;
-    // the descriptor's head (kind, ntasks, layer, ngroups, cur_off, trace_base, gbegin) is
-    // all the hand-out needs; the whole descriptor is copied once a task is taken
-    const OpDesc* gop = P.ops + op;
-    const int4 h1 = __ldg(reinterpret_cast<const int4*>(gop));
-    const int ntasks = h1.y, ng = h1.w > 1 ? h1.w : 1, cur_off = __ldg(&gop->cur_off);
-    const int* gbegin = reinterpret_cast<const int*>(__ldg(reinterpret_cast<const unsigned long long*>(&gop->gbegin)));
-    const int gstart = (int)(((long long)blockIdx.x * ng) / gridDim.x);
-    for (int gi = 0; gi < ng && ok; ++gi) {
-      const int grp = (gstart + gi) % ng;
-      const int lo = gbegin ? __ldg(gbegin + grp) : 0, hi = gbegin ? __ldg(gbegin + grp + 1) : ntasks;
-      unsigned* cur = cursors + cur_off + grp;
-      for (;;) {
-        int tk = 0;
-        if (lane == 0) tk = lo + (int)atomicAdd(cur, 1u);
-        t = __shfl_sync(0xffffffffu, tk, 0);
-        if (t >= hi) break;
-        if (copied != op) {
-          copy_od(S.pod, gop, lane, 32);
-          __syncwarp();
-          copied = op;
-        }
-        const int4 pc = od.pieces ? __ldg(od.pieces + t) : make_int4(0, 0, 0, 0);
-        if (!(ok = push(op, t, pc))) break;
-        tr_first = nullptr;
-        if (P.trace && lane == 0) {  // when the producer took this task
-          const int idx = od.trace_base + t;
-          if (idx < P.trace_cap) {
-            unsigned long long* rec = P.trace + 2 + 6 * (size_t)P.trace_cap + 3 * (size_t)idx;
-            rec[0] = ((unsigned long long)blockIdx.x << 48) | ((unsigned long long)op << 32) | (unsigned)t;
-            rec[1] = globaltimer();
-            tr_first = rec + 2;  // the task's first issued stage stamps it
-          }
-        }
+  while (ok && it.next(op, t)) {
+    if (op != cur) {
+      copy_od(S.pod, P.ops + op, lane, 32);
+      __syncwarp();
+      cur = op;
+    }
+    tr_first = nullptr;
+    if (P.trace && lane == 0) {  // when the producer reached this task
+      const int idx = P.persistent ? it.i - 1 : t;
+      if (idx < P.trace_cap) {
+        unsigned long long* rec = P.trace + 2 + 6 * (size_t)P.trace_cap + 3 * (size_t)idx;
+        rec[0] = ((unsigned long long)blockIdx.x << 48) | ((unsigned long long)op << 32) | (unsigned)t;
+        rec[1] = globaltimer();
+        tr_first = rec + 2;  // the task's first issued stage stamps it
+      }
+    }
     if (od.kind == OP_GEMV) {
       const int tpt = od.tpt > 1 ? od.tpt : 1;
       const bool row_task = od.qc && t == od.ntasks - 1;  // absorb_q's latent-row task streams nothing
       for (int i = 0; i < tpt && ok && !row_task; ++i) {
-      const TaskGeo geo = gemv_geo(od, t * tpt + i, pc);
+      const TaskGeo geo = gemv_geo(od, t * tpt + i);
       const Seg& sg = od.seg[geo.si];
       const uint8_t* base = sg.w;
       if (sg.slot >= 0) {
@@ -1533,8 +1521,8 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
         base += (size_t)m->prod_idx[sg.slot] * sg.w_estride;
       }
       const uint32_t sb = (uint32_t)(od.R * od.kcb);
-      const uint8_t* tile = base + ((size_t)geo.rt * od.nst_total + geo.st0) * sb;
-      for (int st = 0; st < geo.nst && ok; ++st) ok = issue(tile + (size_t)st * sb, sb, nullptr, 0, 0, pol_w);
+      const uint8_t* tile = base + (size_t)(geo.rt * od.S + geo.s) * od.nst * sb;
+      for (int st = 0; st < od.nst && ok; ++st) ok = issue(tile + (size_t)st * sb, sb, nullptr, 0, 0, pol_w);
       }  // units
     } else if (od.kind == OP_ATTN) {
       const int kvh = t / od.nch, c = t % od.nch;
@@ -1583,12 +1571,8 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
         for (int o = 0; o < od.kvl / 256 && ok; ++o) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
       }
     }
-        if (!ok) break;
-      }  // tasks of the group
-    }    // groups
-  }      // ops
-  }      // steps
-  push(-1, -1, make_int4(0, 0, 0, 0));  // end of the consumers' work
+  }
+  }  // steps
   if (lane == 0) m->issued = (int)g;
 }
 
@@ -1626,7 +1610,8 @@ __device__ void signal_loop(const KParams& P, const Smem& S) {
     if (!__shfl_sync(0xffffffffu, ok, 0)) break;
     if (lane == 0) {
       uint32_t end = q + 1;  // batch [q, end)
-      while (end - q < kMail && mbar_try_wait(&m->sig_done[end % kMail], (end / kMail) & 1)) ++end;
+      // a probe of the later slots: test_wait, which never suspends the thread
+      while (end - q < kMail && mbar_test_wait(&m->sig_done[end % kMail], (end / kMail) & 1)) ++end;
       // every consumer write of these tasks happened before their mailbox hand-off
       __threadfence();
       uint32_t i = q;
@@ -1677,37 +1662,32 @@ __device__ void signal_loop(const KParams& P, const Smem& S) {
 template <int WT, bool MLA>
 __device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
   Misc* m = S.m;
-  uint32_t g = 0, q = 0, nmma = 0, qn = 0;
-  int cur = -1;
+  uint32_t g = 0, q = 0, nmma = 0;
+  TaskIter it;
+  it.init(P);
+  int op, t, cur = -1;
   const OpDesc& od = *S.cod;
-  for (;;) {
-    // next task from the producer's queue (thread 0 copies it out and frees the slot)
+  bool stopped = false;
+  for (int step = 0; step < P.n_steps && !stopped; ++step) {
+  if (step > 0) {
+    // the previous step's final op wrote this step's state (see the producer)
     if (threadIdx.x == 0) {
-      const int slot = qn % kTQ;
-      if (mbar_wait(&m->tq_full[slot], (qn / kTQ) & 1, P, &m->abort, cur, -1)) {
-        m->cur_op = m->tq_op[slot];
-        m->cur_t = m->tq_t[slot];
-        m->cur_geo = m->tq_geo[slot];
-        const int4 st = m->tq_st[slot];
-        m->new_step = st.x != m->st.epoch && m->cur_op >= 0;
-        if (m->new_step) {  // a later step of a multi-step launch: its state, nothing cached
-          m->st.epoch = st.x;
-          m->st.pos = st.y;
-          m->st.tok = st.z;
-          m->x_op = -1;
-        }
-        mbar_arrive(&m->tq_empty[slot]);
-      } else {
-        m->cur_op = -1;
+      if (wait_counter(P, P.nops - 1, (unsigned)m->st.epoch, &m->abort, P.nops - 1, 0)) {
+        m->st.epoch = __ldcg(&P.state->epoch);
+        m->st.pos = __ldcg(&P.state->pos);
+        m->st.tok = __ldcg(&P.state->tok);
+        m->st.stop = __ldcg(&P.state->stop);
+        m->x_op = -1;
+        if (!m->st.stop) atomicAdd(P.started, 1u);  // this CTA has read the step's state
       }
     }
-    ++qn;
     if (named_bar_or(1, kConsumers, m->abort)) break;
-    const int op = m->cur_op, t = m->cur_t;
-    const int4 pc = m->cur_geo;
-    if (op < 0) break;
-    if (m->new_step) cur = -1;
-    const unsigned epoch = (unsigned)m->st.epoch;
+    if (m->st.stop) break;
+    it.init(P);
+    cur = -1;
+  }
+  const unsigned epoch = (unsigned)m->st.epoch;
+  while (it.next(op, t)) {
     if (op != cur) {
       copy_od(S.cod, P.ops + op, threadIdx.x, kConsumers);
       if (P.persistent && threadIdx.x == 0) {
@@ -1716,14 +1696,17 @@ __device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
           wait_counter(P, __ldg(&go->dep[1]), epoch, &m->abort, op, t);
       }
       // uniform decision: every consumer thread sees the same value
-      if (named_bar_or(1, kConsumers, m->abort)) break;
+      if (named_bar_or(1, kConsumers, m->abort)) {
+        stopped = true;
+        break;
+      }
       cur = op;
     }
     const uint64_t t_start = P.trace ? globaltimer() : 0;
     if (P.trace && threadIdx.x == 0) m->tr_pro = m->tr_data = t_start;
     const int kind = od.kind;
     if (kind == OP_GEMV) {
-      gemv_consume<WT>(P, od, op, t, S, g, pc);
+      gemv_consume<WT>(P, od, op, t, S, g);
     } else if (kind == OP_FINAL) {
       final_consume(P, od, op, t, S);
     } else {
@@ -1735,9 +1718,13 @@ __device__ __forceinline__ void consumer_loop(const KParams& P, const Smem& S) {
     }
     // A failed wait anywhere in the task makes every thread stop here, after the
     // task's barriers, without publishing the task.
-    if (named_bar_or(1, kConsumers, m->abort)) break;
+    if (named_bar_or(1, kConsumers, m->abort)) {
+      stopped = true;
+      break;
+    }
     post_task(P, m, q++, op, t, t_start);
   }
+  }  // steps
   post_task(P, m, q, -1, -1, 0);  // end sentinel for the signaller
   if (threadIdx.x == 0) m->consumed = (int)g;
 }
@@ -1751,11 +1738,13 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
     m->st = *P.state;
     if (P.tok_in >= 0) m->st.tok = P.tok_in;
     m->abort = 0;
-    m->new_step = 0;
     m->x_op = -1;
     m->x_group = -1;
     m->prod_route_op = -1;
     m->prod_dep_op = -1;
+    // valid expert ids until the router's are read: a task that runs on stale data after
+    // a failed wait (abort) still addresses weights and scales inside their arrays
+    for (int i = 0; i < kMaxTopK; ++i) m->prod_idx[i] = 0;
     m->issued = 0;
     m->consumed = 0;
     for (int i = 0; i < kStages; ++i) {
@@ -1765,10 +1754,6 @@ __global__ void __launch_bounds__(kThreads, 1) engine_kernel(KParams P) {
     for (int i = 0; i < kMail; ++i) {
       mbar_init(&m->sig_done[i], kConsumerWarps);
       mbar_init(&m->sig_free[i], 1);
-    }
-    for (int i = 0; i < kTQ; ++i) {
-      mbar_init(&m->tq_full[i], 1);
-      mbar_init(&m->tq_empty[i], 1);
     }
     mbar_init(&m->mma_bar, 1);
     mbar_init(&m->fin_bar, 1);

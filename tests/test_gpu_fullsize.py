@@ -17,7 +17,7 @@ import torch
 
 import synth
 from oracle import model as om
-from oracle.numerics import argmax_first, bf16_bits_to_f64, margin_topk, rmsnorm, rope, rounder, silu, softmax
+from oracle.numerics import argmax_first, bf16_bits_to_f64, margin_topk, rmsnorm, rope, rounder, silu
 from synth import device as sdev
 from synth import workloads
 
@@ -57,8 +57,8 @@ class Step:
         return np.frombuffer(self.d.dump(self.pkg.dec.DEC_DUMP_OP + i), np.float32).astype(np.float64)
 
     def out(self, layer, name):
-        """The op's output vector (row tiles split among CTAs are already summed on the device)."""
-        return self.raw(self.by_layer[layer][name])
+        i = self.by_layer[layer][name]
+        return self.raw(i).reshape(int(self.plan[i][1]["S"]), -1).sum(0)
 
     def combine(self, layer, name, heads, dim):
         i = self.by_layer[layer][name]
@@ -76,11 +76,17 @@ class Step:
 
 
 def _ffn_out(st, w, l, moe_l):
-    """GPU FFN output of layer l: the dense down projection, or the MoE layer's accumulator (routed
-    experts weighted by the router, plus the shared expert), which the expert-down op dumps."""
+    """GPU FFN output of layer l (dense down sum, or routed + shared experts with router weights)."""
     if w["arch"] == "dense" or l < w["n_dense_layers"]:
         return st.out(l, "down")
-    return st.out(l, "exp_down")
+    d = w["d_model"]
+    r = st.out(l, "router")
+    idx, wts = om.route_topk(r, w["top_k"])
+    dn = st.out(l, "exp_down")
+    f = sum(wts[j] * dn[j * d:(j + 1) * d] for j in range(w["top_k"]))
+    if w["n_shared"]:
+        f = f + dn[w["top_k"] * d:(w["top_k"] + 1) * d]
+    return f
 
 
 @pytest.mark.parametrize("name", ["dense_gqa_bf16_1k", "dense_gqa_fp8_8k", "moe_mla_fp8_1k", "moe_mla_fp8_8k"])
@@ -152,29 +158,22 @@ def test_fullsize_sampled_ops(name):
                 else:
                     r = st.out(l, "router")
                     _cmp(f"L{l} router", r, Wt.mv("router", l, m))
-                    idx, wts = om.route_topk(r, w["top_k"])
+                    idx, _ = om.route_topk(r, w["top_k"])
                     got = st.routes.reshape(-1, w["top_k"])[moe_l]
                     if not np.array_equal(got, idx):
                         assert margin_topk(r, w["top_k"]) < 1e-4, f"L{l}: routes {got} vs {idx}"
-                    # gate|up rows: the shared expert's first, then routed slot j's
                     eh, gu, ref = w["expert_hidden"], st.out(l, "exp_gate|up"), []
-                    ns = 1 if w["n_shared"] else 0
-                    if ns:
-                        ref += [Wt.mv("sh_gate", l, m), Wt.mv("sh_up", l, m)]
                     for e in got:
                         ref += [Wt.mv("exp_gate", l, m, int(e)), Wt.mv("exp_up", l, m, int(e))]
+                    if w["n_shared"]:
+                        ref += [Wt.mv("sh_gate", l, m), Wt.mv("sh_up", l, m)]
                     _cmp(f"L{l} experts gate|up", gu, np.concatenate(ref))
-                    # the layer's FFN output: routed experts weighted by the GPU's router weights
-                    # (renormalised softmax of its logits), plus the shared expert
-                    ref = np.zeros(d)
-                    gsl = lambda j: (gu[2 * j * eh:(2 * j + 1) * eh], gu[(2 * j + 1) * eh:(2 * j + 2) * eh])
-                    if ns:
-                        g_, u_ = gsl(0)
-                        ref += Wt.mv("sh_down", l, R(silu(g_) * u_))
-                    for j, e in enumerate(got):
-                        g_, u_ = gsl(ns + j)
-                        ref += wts[j] * Wt.mv("exp_down", l, R(silu(g_) * u_), int(e))
-                    _cmp(f"L{l} experts down", st.out(l, "exp_down"), ref)
+                    dn, ref = st.out(l, "exp_down"), []
+                    for j, e in enumerate(list(got) + ([-1] if w["n_shared"] else [])):
+                        g_, u_ = gu[2 * j * eh:(2 * j + 1) * eh], gu[(2 * j + 1) * eh:(2 * j + 2) * eh]
+                        nm = ("sh_down", -1) if e < 0 else ("exp_down", int(e))
+                        ref.append(Wt.mv(nm[0], l, R(silu(g_) * u_), nm[1]))
+                    _cmp(f"L{l} experts down", dn, np.concatenate(ref))
             if w["arch"] != "dense" and l >= w["n_dense_layers"]:
                 moe_l += 1
             h = h + _ffn_out(st, w, l, moe_l)

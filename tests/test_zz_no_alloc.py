@@ -56,13 +56,14 @@ def test_noalloc_attention_matches_decode_step():
         d.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
         plan = [line.split() for line in d.plan_text().splitlines()[:-1]]
         assert plan[0][1] == "qkv" and plan[1][1] == "attn"
+        S = int(dict(f.split("=") for f in plan[0][2:] if "=" in f)["S"])
         nch = int(dict(f.split("=") for f in plan[1][2:] if "=" in f)["nch"])
         tok = 5
         for call in range(2):
             pos = w["ctx"] + call
             tok = d.step(tok)
             # the step's attention inputs: q of layer 0 (RoPE at pos, rounded to bf16) ...
-            qkv = np.frombuffer(d.dump(pkg.dec.DEC_DUMP_OP + 0), np.float32).astype(np.float64)
+            qkv = np.frombuffer(d.dump(pkg.dec.DEC_DUMP_OP + 0), np.float32).astype(np.float64).reshape(S, -1).sum(0)
             qr = qkv[: hq * hd].reshape(hq, hd)
             half = hd // 2
             ang = pos * w["rope_theta"] ** (-2.0 * np.arange(half) / hd)
