@@ -257,6 +257,25 @@ def run_ours(args, rank, world, local_rank):
             ablation[name] = {"ms_per_step": ms / args.steps, "tokens_per_s": args.steps / (ms / 1e3)}
         ablation["persistent"] = {"ms_per_step": ms_main / args.steps, "tokens_per_s": args.steps / (ms_main / 1e3)}
         dec.set_exec_mode(pkg.dec.DEC_PERSISTENT)
+        # one launch for the whole generation: dec_generate_async runs args.steps steps in a single
+        # persistent kernel (greedy feedback and the token ring on the device)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        for timed in (False, True):
+            dec.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])
+            if dist is not None:
+                dist.barrier()
+            if timed:
+                ev[0].record(stream)
+            dec.generate_async(first, args.steps)
+            if timed:
+                ev[1].record(stream)
+            got = dec.generate_wait(args.steps)
+            torch.cuda.synchronize()
+            if len(got) != args.steps:
+                raise RuntimeError(f"generation ended after {len(got)} of {args.steps} steps")
+        ms = max_over_ranks(ev[0].elapsed_time(ev[1]), dist)
+        ablation["generation_one_launch"] = {"ms_per_step": ms / args.steps, "tokens_per_s": args.steps / (ms / 1e3),
+                                             "launches": 1, "steps": args.steps}
 
     # e2e: the synchronous public call, token in from the host, greedy token out to the host
     dec.set_kv_cache(k.data_ptr(), v.data_ptr(), w["ctx"])

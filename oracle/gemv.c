@@ -68,3 +68,61 @@ void oracle_gemv_fp8(const uint8_t* q, const float* s, int64_t N, int64_t K, con
     y[n] = acc;
   }
 }
+
+/*
+ * Float32-accumulation twins.  NOT the definition: the same products, summed
+ * in a float32 accumulator per 128-column block and the blocks then added in
+ * float32, as an implementation that accumulates in float32 would.  Tests use
+ * them only to measure how far such an implementation can land from the
+ * float64 definition on a chaotic random-init model (a calibration of the
+ * end-to-end tolerance); no expected value is ever taken from them.
+ */
+void oracle_gemv_f32_acc32(const float* W, int64_t N, int64_t K, const double* x, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    const float* w = W + n * K;
+    float acc = 0.f;
+    for (int64_t k0 = 0; k0 < K; k0 += 128) {
+      float part = 0.f;
+      for (int64_t k = k0; k < K && k < k0 + 128; ++k) part += w[k] * (float)x[k];
+      acc += part;
+    }
+    y[n] = acc;
+  }
+}
+
+void oracle_gemv_bf16_acc32(const uint16_t* W, int64_t N, int64_t K, const double* x, double* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    const uint16_t* w = W + n * K;
+    float acc = 0.f;
+    for (int64_t k0 = 0; k0 < K; k0 += 128) {
+      float part = 0.f;
+      for (int64_t k = k0; k < K && k < k0 + 128; ++k) {
+        uint32_t u = (uint32_t)w[k] << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        part += f * (float)x[k];
+      }
+      acc += part;
+    }
+    y[n] = acc;
+  }
+}
+
+void oracle_gemv_fp8_acc32(const uint8_t* q, const float* s, int64_t N, int64_t K, const double* table,
+                           const double* x, double* y) {
+  const int64_t nbc = (K + 127) / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* w = q + n * K;
+    const float* srow = s + (n / 128) * nbc;
+    float acc = 0.f;
+    for (int64_t b = 0; b < nbc; ++b) {
+      float part = 0.f;
+      for (int64_t k = b * 128; k < K && k < b * 128 + 128; ++k) part += (float)table[w[k]] * (float)x[k];
+      acc += part * srow[b];
+    }
+    y[n] = acc;
+  }
+}

@@ -44,6 +44,9 @@ def lib():
         L.oracle_gemv_f32.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_gemv_bf16.argtypes = [vp, i64, i64, vp, vp]
         L.oracle_gemv_fp8.argtypes = [vp, vp, i64, i64, vp, vp, vp]
+        L.oracle_gemv_f32_acc32.argtypes = [vp, i64, i64, vp, vp]
+        L.oracle_gemv_bf16_acc32.argtypes = [vp, i64, i64, vp, vp]
+        L.oracle_gemv_fp8_acc32.argtypes = [vp, vp, i64, i64, vp, vp, vp]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
         L.oracle_get_threads.restype = ctypes.c_int
         _lib = L
@@ -75,6 +78,26 @@ def gemv(t: dict, x: np.ndarray) -> np.ndarray:
     else:
         lib().oracle_gemv_fp8(d.ctypes.data, t["scales"].ctypes.data, N, K, _TABLE.ctypes.data, x.ctypes.data,
                               y.ctypes.data)
+    return y
+
+
+def gemv_acc32(t: dict, x: np.ndarray) -> np.ndarray:
+    """Float32-accumulation twin of gemv: NOT the definition.  The same products summed in
+    float32 (per 128-column block, then across blocks), as a float32-accumulating
+    implementation would.  Tests swap it in for gemv only to measure how far such an
+    implementation lands from the float64 definition on a chaotic random-init model."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    N, K = t["data"].shape
+    assert x.shape == (K,), (x.shape, K)
+    y = np.empty(N, dtype=np.float64)
+    d = t["data"]
+    if t["dtype"] == "f32":
+        lib().oracle_gemv_f32_acc32(d.ctypes.data, N, K, x.ctypes.data, y.ctypes.data)
+    elif t["dtype"] == "bf16":
+        lib().oracle_gemv_bf16_acc32(d.ctypes.data, N, K, x.ctypes.data, y.ctypes.data)
+    else:
+        lib().oracle_gemv_fp8_acc32(d.ctypes.data, t["scales"].ctypes.data, N, K, _TABLE.ctypes.data,
+                                    x.ctypes.data, y.ctypes.data)
     return y
 
 

@@ -54,11 +54,8 @@ def _brute_gemv(Wv, x):
     return np.array([sum(float(Wv[n, k]) * float(x[k]) for k in range(Wv.shape[1])) for n in range(Wv.shape[0])])
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8"])
-def test_gemv_against_brute_force(dtype):
-    rng = np.random.default_rng(3)
-    N, K = 260, 300  # ragged against the 128-blocks
-    x = rng.normal(size=K)
+def _gemv_case(dtype, rng, N, K):
+    """A host weight of `dtype` and its float64 value."""
     if dtype == "f32":
         data = rng.normal(size=(N, K)).astype(np.float32)
         t = dict(dtype="f32", data=data, scales=None)
@@ -76,9 +73,36 @@ def test_gemv_against_brute_force(dtype):
         for n in range(N):
             for k in range(K):
                 Wv[n, k] = nm.e4m3_value(int(q[n, k])) * float(s[n // 128, k // 128])
+    return t, Wv
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8"])
+def test_gemv_against_brute_force(dtype):
+    rng = np.random.default_rng(3)
+    N, K = 260, 300  # ragged against the 128-blocks
+    x = rng.normal(size=K)
+    t, Wv = _gemv_case(dtype, rng, N, K)
     y = om.gemv(t, x)
     ref = _brute_gemv(Wv, x)
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "fp8"])
+def test_gemv_acc32_twin_is_float32_summation(dtype):
+    """The float32-accumulation twin (a tolerance calibration, not the definition) stays within the
+    textbook bound of float32 recursive summation, |y - y_exact| <= gamma_{K+2} * sum|w x| with
+    gamma_n = n u / (1 - n u), u = 2^-24, and really does round in float32 (not bit-equal to float64)."""
+    rng = np.random.default_rng(5)
+    N, K = 260, 300
+    x = rng.normal(size=K).astype(np.float32).astype(np.float64)  # activations are float32-exact
+    t, Wv = _gemv_case(dtype, rng, N, K)
+    y = om.gemv_acc32(t, x)
+    ref = _brute_gemv(Wv, x)
+    u = 2.0 ** -24
+    gamma = (K + 2) * u / (1 - (K + 2) * u)
+    assert np.all(np.abs(y - ref) <= gamma * (np.abs(Wv) @ np.abs(x)))
+    assert np.any(y != ref)
+    assert np.all(y.astype(np.float32).astype(np.float64) == y)
 
 
 def test_fp8_block_dequant_against_scalar_definition():
