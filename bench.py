@@ -53,9 +53,11 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per step of the engine kernel from the committed ncu summary, if it matches this source."""
-    p = os.path.join(ROOT, "profiles", f"engine_kernel_{workload}.json")
+def recorded_traffic(bytes_step: float):
+    """DRAM bytes per step of the engine kernel, scaled from the committed ncu record of the one-layer
+    profiling case (its traffic / algorithmic-bytes ratio times this workload's algorithmic bytes),
+    if the record was taken on this kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "engine_kernel_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -65,7 +67,7 @@ def recorded_traffic(workload: str):
     valid = {d.get("source_hash")} | {x["source_hash"] for x in d.get("same_kernel_sources", [])}
     if source_hash() not in valid:
         return None
-    return d.get("dram_bytes_per_step")
+    return bytes_step * d["dram_bytes_per_step"] / d["algorithmic_bytes_per_step"]
 
 
 class ClockSampler:
@@ -318,7 +320,7 @@ def run_ours(args, rank, world, local_rank):
                 "l2": l2_note(bytes_step)},
             "achieved_hbm_gbs": achieved,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                         "frac": achieved / peak, "traffic": recorded_traffic(bytes_step),
                          "bytes_per_step": bytes_step, "frac_of_8tbs": achieved / 8000.0,
                          "kernel": "engine_kernel (one persistent launch per step)"},
             "clocks": clk,

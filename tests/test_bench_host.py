@@ -37,33 +37,35 @@ def test_clock_summary_without_samples_says_unavailable():
     assert _summary([]) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
 
 
-@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(ROOT, "profiles", "engine_kernel_*.json"))))
-def test_traffic_records_are_consistent(path):
-    """Each committed DRAM record: read + write = per-step traffic; its algorithmic bytes are the
-    workload's active bytes at the captured step (context + 3 warm-up steps + half of 2 timed
-    steps, as its command runs it); traffic exceeds them by less than 1 %."""
-    with open(path) as f:
+TRAFFIC = os.path.join(ROOT, "profiles", "engine_kernel_traffic.json")
+
+
+def test_traffic_record_is_consistent():
+    """The committed DRAM record of the one-layer profiling case: read + write = per-step traffic;
+    its algorithmic bytes are the workload's active bytes at the captured step (context + 3
+    warm-up steps + half of 2 timed steps, as its command runs it); traffic exceeds them by
+    less than 2 %."""
+    with open(TRAFFIC) as f:
         d = json.load(f)
     assert d["dram_bytes_read"] + d["dram_bytes_write"] == d["dram_bytes_per_step"]
     w = workloads.get(d["workload"])
     assert "--steps 2 --warmup 3" in d["command"] and "--clock-control none" in d["command"]
+    assert f"--workload {d['workload']}" in d["command"]
     assert workloads.active_bytes_per_token(w, w["ctx"] + 4)["total"] == d["algorithmic_bytes_per_step"]
-    assert 1.0 <= d["dram_bytes_per_step"] / d["algorithmic_bytes_per_step"] < 1.01
+    assert 1.0 <= d["dram_bytes_per_step"] / d["algorithmic_bytes_per_step"] < 1.02
 
 
 def test_recorded_traffic_needs_the_matching_source(monkeypatch):
-    recs = glob.glob(os.path.join(ROOT, "profiles", "engine_kernel_*.json"))
-    assert recs
-    with open(recs[0]) as f:
+    with open(TRAFFIC) as f:
         d = json.load(f)
+    ratio = d["dram_bytes_per_step"] / d["algorithmic_bytes_per_step"]
     monkeypatch.setattr(bench, "source_hash", lambda: d["source_hash"])
-    assert bench.recorded_traffic(d["workload"]) == d["dram_bytes_per_step"]
+    assert bench.recorded_traffic(8e9) == pytest.approx(8e9 * ratio)
     for x in d.get("same_kernel_sources", []):
         monkeypatch.setattr(bench, "source_hash", lambda: x["source_hash"])
-        assert bench.recorded_traffic(d["workload"]) == d["dram_bytes_per_step"]
+        assert bench.recorded_traffic(8e9) == pytest.approx(8e9 * ratio)
     monkeypatch.setattr(bench, "source_hash", lambda: "0" * 16)
-    assert bench.recorded_traffic(d["workload"]) is None
-    assert bench.recorded_traffic("no_such_workload") is None
+    assert bench.recorded_traffic(8e9) is None
 
 
 def test_peak_fallback_without_measured_file(monkeypatch, tmp_path):
