@@ -228,32 +228,28 @@ __device__ __forceinline__ void store_x4(uint8_t* work, int in_bf16, int e, floa
   }
 }
 
-// Softmax top-k router (one warp, all 32 lanes call): pick the k largest logits,
+// Router logits: sum of the S split-K partials of each of E experts, in split order, one
+// expert per consumer thread (its S loads in flight together).  Out of line: it runs once per
+// MoE layer and must not add to the register budget of the hot loops.
+__device__ __noinline__ void router_sum(const float* out, int S, int stride, int E, float* dst) {
+  for (int e = threadIdx.x; e < E; e += kConsumers) {
+    float v = 0.f;
+    for (int s0 = 0; s0 < S; ++s0) v += ldcg(out + (size_t)s0 * stride + e);
+    dst[e] = v;
+  }
+}
+
+// Softmax top-k router (one warp, all 32 lanes call) over E <= 256 summed logits in
+// shared memory: pick the k largest logits,
 // ties to the lower expert id, weights renormalised over the chosen k:
 // w_j = exp(r_j - r_max) / sum_i exp(r_i - r_max).  Returns false (every lane) if
 // any logit is NaN or infinite; the ids and weights are then still written.
-__device__ __forceinline__ bool warp_route(const PSet& logits, int E, int k, int* idx_out, float* w_out) {
+__device__ __forceinline__ bool warp_route(const float* logits, int E, int k, int* idx_out, float* w_out) {
   const int lane = threadIdx.x & 31;
   float v[8];
   int taken = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = 0.f;
-  // sum the split-K partials, 4 splits x 8 logits = 32 independent loads per batch
-  const float* base = logits.ptr + logits.off;
-  for (int s0 = 0; s0 < logits.S; s0 += 4) {
-    float u[4][8];
-#pragma unroll
-    for (int ds = 0; ds < 4; ++ds)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        u[ds][i] = (s0 + ds < logits.S && e < E) ? ldcg(base + (size_t)(s0 + ds) * logits.stride + e) : 0.f;
-      }
-#pragma unroll
-    for (int ds = 0; ds < 4; ++ds)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] += u[ds][i];
-  }
+  for (int i = 0; i < 8; ++i) v[i] = lane + 32 * i < E ? logits[lane + 32 * i] : 0.f;
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -567,9 +563,19 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   return ((unsigned long long)u << 32) | (0xFFFFFFFFu - (uint32_t)idx);
 }
 
-template <int WT>
-__device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* x, int k0, int kcb, int G, int rpt,
-                                           int c, int rg, float scale, float* acc) {
+// This thread's 16-byte chunks of a ring stage: chunk c of rows rg, rg + G, ... (rpt rows).
+// They are taken into registers first so that the stage can go back to the producer before
+// the arithmetic: the slot's next copy then overlaps this stage's compute.
+template <int RPT>
+__device__ __forceinline__ void gemv_load(const uint8_t* stage, int kcb, int G, int rpt, int c, int rg, uint4* wv) {
+#pragma unroll
+  for (int i = 0; i < RPT; ++i)
+    if (i < rpt) wv[i] = *reinterpret_cast<const uint4*>(stage + (rg + G * i) * kcb + c * 16);
+}
+
+template <int WT, int RPT>
+__device__ __forceinline__ void gemv_stage(const uint4* wv, const uint8_t* x, int k0, int rpt, int c, float scale,
+                                           float* acc) {
   if constexpr (WT == WT_FP8) {
     const uint4* xv = reinterpret_cast<const uint4*>(x + 2 * (k0 + c * 16));
     const uint4 xa = xv[0], xb = xv[1];
@@ -581,11 +587,9 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
       xf[2 * i + 1] = bf16hi(xw[i]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < RPT; ++i) {
       if (i >= rpt) break;
-      const int r = rg + G * i;
-      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * kcb + c * 16);
-      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
       float part = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -608,11 +612,9 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
       xf[2 * i + 1] = bf16hi(xw[i]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < RPT; ++i) {
       if (i >= rpt) break;
-      const int r = rg + G * i;
-      const uint4 wv = *reinterpret_cast<const uint4*>(stage + r * kcb + c * 16);
-      const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+      const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
       float a = acc[i];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -624,15 +626,15 @@ __device__ __forceinline__ void gemv_stage(const uint8_t* stage, const uint8_t* 
   } else {
     const float4 xa = *reinterpret_cast<const float4*>(x + 4 * (k0 + c * 4));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < RPT; ++i) {
       if (i >= rpt) break;
-      const int r = rg + G * i;
-      const float4 wv = *reinterpret_cast<const float4*>(stage + r * kcb + c * 16);
+      const float4 w4 = make_float4(__uint_as_float(wv[i].x), __uint_as_float(wv[i].y), __uint_as_float(wv[i].z),
+                                    __uint_as_float(wv[i].w));
       float a = acc[i];
-      a = fmaf(wv.x, xa.x, a);
-      a = fmaf(wv.y, xa.y, a);
-      a = fmaf(wv.z, xa.z, a);
-      a = fmaf(wv.w, xa.w, a);
+      a = fmaf(w4.x, xa.x, a);
+      a = fmaf(w4.y, xa.y, a);
+      a = fmaf(w4.z, xa.z, a);
+      a = fmaf(w4.w, xa.w, a);
       acc[i] = a;
     }
   }
@@ -673,8 +675,10 @@ __device__ __forceinline__ void gemv_task(const KParams& P, const OpDesc& od, in
       const int cb = (k0 + c * 16) >> 7;
       scale = cb < nkb ? __ldg(sc + cb) : 0.f;
     }
-    gemv_stage<WT>(stage, S.work, k0, KCB, G, RPT, c, rg, scale, acc);
+    uint4 wv[RPT];
+    gemv_load<RPT>(stage, KCB, G, RPT, c, rg, wv);
     release_stage(S, g);
+    gemv_stage<WT, RPT>(wv, S.work, k0, RPT, c, scale, acc);
     ++g;
   }
   // reduce the CPR partials of every row
@@ -820,10 +824,15 @@ __device__ __forceinline__ void gemv_consume(const KParams& P, const OpDesc& od,
       m->last_task = prev + 1 == (unsigned)m->st.epoch * (unsigned)od.ntasks;
     }
     named_bar_sync(1, kConsumers);
-    if (m->last_task && threadIdx.x < 32) {
+    if (m->last_task) {
       __threadfence();
-      if (!warp_route(PSet{od.out, od.S, od.out_stride, 0}, od.n_experts, od.top_k, od.rt_ids, od.rt_w) &&
-          threadIdx.x == 0)
+      // every consumer thread sums one expert's split-K partials, in split order (all of them
+      // in flight at once); one warp then takes the top-k from shared memory
+      router_sum(od.out, od.S, od.out_stride, od.n_experts, m->red);
+      named_bar_sync(1, kConsumers);
+    }
+    if (m->last_task && threadIdx.x < 32) {
+      if (!warp_route(m->red, od.n_experts, od.top_k, od.rt_ids, od.rt_w) && threadIdx.x == 0)
         report_nonfinite(P, op, t);
       if (od.route_dump && threadIdx.x < od.top_k) od.route_dump[threadIdx.x] = __ldcg(od.rt_ids + threadIdx.x);
     }
