@@ -219,7 +219,12 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("steps + warmup must fit the workload's decode length")
     dec = pkg.Decoder(pkg.config_from_workload(w, device=local_rank))
     sdev.load_weights(dec, w)
-    k, v = sdev.synthetic_cache_device(w)
+    t_pf = time.perf_counter()
+    if args.cache == "prefill":  # the context decoded on the GPU from its token ids (untimed setup)
+        k, v = sdev.prefill_by_decode(dec, w, device=f"cuda:{local_rank}")
+    else:
+        k, v = sdev.synthetic_cache_device(w, device=f"cuda:{local_rank}")
+    t_pf = time.perf_counter() - t_pf
     first = int(synth.tokens(w["seed"], synth.TOKENS_FIRST, 1, w["vocab"])[0])
     stream = torch.cuda.Stream()
     dec.set_stream(stream.cuda_stream)
@@ -313,7 +318,9 @@ def run_ours(args, rank, world, local_rank):
             "vs_baseline": None,
             "dtype": "fp8-e4m3 weights (128x128 block scales), bf16 activations, fp32 accumulate"
             if w["weight_dtype"] == "fp8" else w["weight_dtype"],
-            "data": "synthetic: seeded random-init weights of the named shape, seeded random prefilled cache",
+            "data": "synthetic: seeded random-init weights of the named shape; " + (
+                f"context of {w['ctx']} seeded uniform-random token ids decoded on the GPU from an empty cache "
+                f"({t_pf:.1f} s, untimed)" if args.cache == "prefill" else "seeded random cache draw"),
             "config": {"workload": args.workload, "context": w["ctx"], "decode_positions": [
                 w["ctx"] + args.warmup, w["ctx"] + args.warmup + args.steps], "users": world,
                 "parallelism": f"replicas{world}", "exec_mode": "persistent",
@@ -343,6 +350,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=64)
     ap.add_argument("--no-ablation", dest="ablation", action="store_false")
+    ap.add_argument("--cache", choices=("prefill", "synthetic"), default="prefill",
+                    help="context cache: decoded on the GPU from the workload's context ids (default), "
+                         "or drawn directly from the seeded generator")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget-s", type=float, default=30.0)
     args = ap.parse_args()

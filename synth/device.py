@@ -78,3 +78,39 @@ def host_cache_arrays(w, parts: dict):
             t = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)
             out.append(t.view(torch.int16).numpy().copy())
     return out
+
+
+def context_ids(w, n=None):
+    """The workload's context: n (default ctx) seeded uniform-random token ids."""
+    from . import TOKENS_CONTEXT, tokens
+
+    return tokens(w["seed"], TOKENS_CONTEXT, w["ctx"] if n is None else n, w["vocab"])
+
+
+def prefill_by_decode(d, w, n=None, device="cuda"):
+    """Fill decoder d's cache with a real context: from an empty cache, the GPU decodes the
+    workload's first n context ids (default ctx), one step per id, each fed from the host.
+
+    Returns the cache as device tensors in the layout dec_set_kv_cache takes (dense (k, v),
+    MLA (latent, pe); the cache dtype's bits), so that it can be installed again later.
+    The decoder is left at position n."""
+    ids = context_ids(w, n)
+    d.set_kv_cache(0, 0, 0)
+    for t in ids:
+        d.step_async(int(t))
+    d.sync()
+    raw = np.frombuffer(d.dump(_dump_kv()), np.uint8)
+    if w["arch"] == "dense":
+        first = raw.size // 2  # K then V, equal sizes
+    else:  # latent [L][n][kv_lora] then pe [L][n][rope]
+        first = raw.size * w["kv_lora"] // (w["kv_lora"] + w["qk_rope"])
+    el = torch.float32 if workloads.act_dtype(w) == "f32" else torch.int16
+    a = torch.from_numpy(raw[:first].copy()).view(el).to(device)
+    b = torch.from_numpy(raw[first:].copy()).view(el).to(device)
+    return a, b
+
+
+def _dump_kv():
+    from persistent_sm_decode_02_b200 import dec
+
+    return dec.DEC_DUMP_KV
