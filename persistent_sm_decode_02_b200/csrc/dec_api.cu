@@ -1348,6 +1348,13 @@ static KParams kparams(dec_ctx* c, int persistent, int op, int tok_in) {
   P.trace_cap = c->trace_cap;
   P.tok_in = tok_in;
   P.test_stall = (c->cfg.flags & DEC_FLAG_TEST_STALL) ? 1 : 0;
+  {
+    // cache bytes one step reads at the current position (all layers), against 3/4 of L2
+    const dec_config& f = c->cfg;
+    const long long row = f.arch == DEC_ARCH_MLA_MOE ? (long long)(f.kv_lora + f.qk_rope) * c->eb
+                                                     : 2LL * f.n_kv_heads * f.head_dim * c->eb;
+    P.kv_evict_first = (long long)(c->pos + 1) * f.n_layers * row > kL2Bytes / 4 * 3 ? 1 : 0;
+  }
   P.n_steps = 1;
   P.gen = c->d_gen;
   P.tok_count = reinterpret_cast<unsigned*>(c->d_map);

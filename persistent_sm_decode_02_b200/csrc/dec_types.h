@@ -17,6 +17,7 @@ constexpr int kConsumers = kConsumerWarps * 32;  // threads that compute
 constexpr int kThreads = kConsumers + 64;        // + one producer warp (streams weights) + one signaller warp
 constexpr int kStageBytes = 32768;               // one ring stage
 constexpr int kStages = 5;                       // ring depth (160 KB in flight per SM)
+constexpr long long kL2Bytes = 126LL << 20;      // L2 of one GPU (both dies)
 constexpr int kWorkBytes = 48 * 1024;            // per-task scratch (input vector / attention state)
 constexpr int kCombineOff = 40 * 1024;           // split-KV combine weights inside the scratch (<= 2048 floats)
 constexpr int kMaxCombine = (kWorkBytes - kCombineOff) / 4;
@@ -200,6 +201,8 @@ struct KParams {
   int trace_cap;
   int tok_in;                 // >= 0: token of this step given by the host; < 0: the state's token
   int test_stall;             // failure-path test: never publish task 0 of op 0
+  int kv_evict_first;         // 1: cache reads take the L2 evict-first policy (the caches a step reads exceed
+                              // what L2 could keep for the next step), 0: evict-last (they are re-read from L2)
   // ---- generation: a whole decode lifetime in one launch (persistent mode, n_steps > 1)
   int n_steps;                // steps this launch runs (1: one step)
   const GenState* gen;        // device: the running generation, if any

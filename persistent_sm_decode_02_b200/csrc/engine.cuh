@@ -1433,7 +1433,9 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
   Misc* m = S.m;
   const int lane = threadIdx.x & 31;
   const uint64_t pol_w = policy_evict_first();  // weights: streamed once per step
-  const uint64_t pol_kv = policy_evict_last();  // caches: re-read every step
+  // caches: re-read every step, so kept in L2 while they fit there; past that they only push
+  // other lines out and are streamed like the weights
+  const uint64_t pol_kv = P.kv_evict_first ? policy_evict_first() : policy_evict_last();
   uint32_t g = 0;
   TaskIter it;
   it.init(P);
