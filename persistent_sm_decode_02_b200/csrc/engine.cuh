@@ -1196,9 +1196,10 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   Misc* m = S.m;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int pos = m->st.pos, T = pos + 1, nch = od.nch, H = od.H;
-  const int c = t, t0 = c * kMlaBlock;
+  const int os = od.osplit > 1 ? od.osplit : 1, part = t % os;  // part: which half of O's columns
+  const int c = t / os, t0 = c * kMlaBlock;
   if (t0 >= T) {  // block beyond the sequence: empty partial (l = 0)
-    for (int h = tid; h < H; h += kConsumers) {
+    for (int h = tid; h < H && part == 0; h += kConsumers) {
       od.m_out[(size_t)h * nch + c] = -INFINITY;
       od.l_out[(size_t)h * nch + c] = 0.f;
     }
@@ -1278,7 +1279,7 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     fence_async_smem();
     tc_fence_before();
     named_bar_sync(1, kConsumers);
-    if (half == 0 && h < H) {  // (m, l) in natural-log units for the combine
+    if (half == 0 && h < H && part == 0) {  // (m, l) in natural-log units for the combine
       od.m_out[(size_t)h * nch + c] = mx * 0.6931471805599453f;  // log2 units -> natural log
       od.l_out[(size_t)h * nch + c] = red[h] + red[128 + h];
     }
@@ -1286,6 +1287,7 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   // ---- O = P . C_lat over kvl / 256 stages (hi and lo parts of P)
   const int nks = (n + 15) / 16;
   for (int o = 0; o < kvl / 256; ++o) {
+    if (os > 1 && o != part) continue;  // the other half of the columns is the other task's
     wait_full(P, S, g, op, t);
     uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
     if (warp == 0) {
@@ -1305,15 +1307,17 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
     ++g;
   }
   if (tid == 0) tc_commit(&m->mma_bar);
-  // ---- epilogue: warp w reads lanes 32 (w % 4).. and columns 256 (w / 4)..; each
+  // ---- epilogue: warp w reads lanes 32 (w % 4).. and columns col0.. (its half of the
+  // task's columns); each
   // 32 x 32 tile goes through shared memory so that the stores are coalesced
   mbar_wait(&m->mma_bar, (nmma + 1) & 1, P, &m->abort, op, t);
   __syncwarp();
   tc_fence_after();
-  const int col0 = 256 * half;
+  // all 512 columns (256 per warp half), or this task's 256 (128 per warp half)
+  const int ncc = os > 1 ? 4 : 8, col0 = os > 1 ? 256 * part + 128 * half : 256 * half;
   float* tile = reinterpret_cast<float*>(S.work) + warp * (32 * 36);  // [32 heads][36] (P is dead)
 #pragma unroll 1
-  for (int cc = 0; cc < 8; ++cc) {
+  for (int cc = 0; cc < ncc; ++cc) {
     uint32_t r[32];
     tmem_ld32(tm + ((uint32_t)(32 * quad) << 16) + col0 + 32 * cc, r);
     tmem_wait_ld();
@@ -1546,10 +1550,12 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
                    od.np * rowb, pol_kv);
       }
     } else if (od.kind == OP_MLA) {
-      // block t: nine (Q chunk, C chunk) stages for S, then two C stages for O
-      if (t * kMlaBlock <= pos) {
+      // block cb: nine (Q chunk, C chunk) stages for S, then two C stages for O (one: the
+      // task's half of O's columns when the op splits O)
+      const int os = od.osplit > 1 ? od.osplit : 1, cb = t / os, part = t % os;
+      if (cb * kMlaBlock <= pos) {
         const int rowe = od.kvl + od.rdim, nS = rowe / 64;
-        const uint8_t* blk = (const uint8_t*)od.kcache + (size_t)t * rowe * kMlaBlock * 2;
+        const uint8_t* blk = (const uint8_t*)od.kcache + (size_t)cb * rowe * kMlaBlock * 2;
         const uint8_t* q = (const uint8_t*)od.qc;
         int early = 0;
         const uint32_t g0 = g;
@@ -1557,7 +1563,7 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
           // The cache chunks do not depend on this step's ops (except in the block that
           // absorb_q appends to): start them in the first free stages now; the query
           // chunks (written by absorb_q) join the same stages once absorb_q is done.
-          if (pos >= (t + 1) * kMlaBlock)
+          if (pos >= (cb + 1) * kMlaBlock)
             for (; early < nS && early < kStages && ok; ++early)
               ok = issue(nullptr, 16384, blk + early * 8192, 8192, 16384, pol_kv);  // expects both parts
           int r = ok ? 1 : 0;
@@ -1579,7 +1585,8 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
           __syncwarp();
         }
         for (int j = early; j < nS && ok; ++j) ok = issue(q + j * 16384, 16384, blk + j * 8192, 8192, 16384, pol_kv);
-        for (int o = 0; o < od.kvl / 256 && ok; ++o) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
+        for (int o = 0; o < od.kvl / 256 && ok; ++o)
+          if (os == 1 || o == part) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
       }
     }
   }
