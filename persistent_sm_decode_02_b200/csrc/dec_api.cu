@@ -609,9 +609,9 @@ static int build_plan(dec_ctx* c) {
         a.rdim = rd;
         a.nope = nope;
         a.nch = nch_mla;
-        // few blocks (short caches): two tasks per block, each with half of O's columns, so
-        // that the per-task output half goes to twice the CTAs
-        a.osplit = 2 * nch_mla <= c->n_ctas && kvl % 512 == 0 ? 2 : 1;
+        // few blocks (short caches): two or four tasks per block, each with that share of O's
+        // columns, so that the output work goes to more CTAs
+        a.osplit = kvl != 512 ? 1 : 4 * nch_mla <= c->n_ctas ? 4 : 2 * nch_mla <= c->n_ctas ? 2 : 1;
         a.ntasks = nch_mla * a.osplit;
         a.qc = qc;
         a.ckv = PSet{p1.out, p1.S, p1.out_stride, f.q_lora};

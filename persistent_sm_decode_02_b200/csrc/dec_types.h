@@ -152,7 +152,7 @@ struct alignas(16) OpDesc {
   float* o_fin;  // dense: combined attention output [hq][hd] (the last chunk task of a kv head writes it;
                  // `fin` then holds one finished-task counter per kv head)
   int np;  // positions per ring stage
-  int osplit;  // MLA: tasks per cache block (2: each computes S and half of O's 512 latent columns)
+  int osplit;  // MLA: tasks per cache block (1, 2 or 4: each computes S and that share of O's columns)
   // ---- final op
   const unsigned long long* fin_best;
   int fin_n;

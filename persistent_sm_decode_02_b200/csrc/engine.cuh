@@ -1212,6 +1212,7 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   const uint32_t tm = m->tmem;
   constexpr uint32_t kIdS = umma_idesc_bf16(128, kMlaBlock, false);
   constexpr uint32_t kIdO = umma_idesc_bf16(128, 256, true);
+  constexpr uint32_t kIdO4 = umma_idesc_bf16(128, 128, true);  // a quarter of the columns
   // ---- S = Q . C^T over (kvl + rd) / 64 stages
   const int nS = rowe / 64;
   for (int j = 0; j < nS; ++j) {
@@ -1286,17 +1287,19 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   }
   // ---- O = P . C_lat over kvl / 256 stages (hi and lo parts of P)
   const int nks = (n + 15) / 16;
-  for (int o = 0; o < kvl / 256; ++o) {
-    if (os > 1 && o != part) continue;  // the other half of the columns is the other task's
+  for (int o = 0; o < (os == 4 ? 1 : kvl / 256); ++o) {
+    if (os == 2 && o != part) continue;  // the other half of the columns is the other task's
     wait_full(P, S, g, op, t);
     uint8_t* stage = S.ring + (g % kStages) * kStageBytes;
     if (warp == 0) {
       if (lane == 0) {
         tc_fence_after();
+        // TMEM columns of this stage's O: 256 o (halves), 128 part (quarters)
+        const uint32_t dcol = os == 4 ? 128 * part : 256 * o;
         for (int s = 0; s < nks; ++s) {  // K = 16 positions
           const uint64_t b = umma_desc(stage + s * 256, 128, 1024);  // MN-major: K step 128 B, N step 1024 B
-          tc_mma(tm + 256 * o, umma_desc(Phi + s * 4096, 2048, 128), b, kIdO, s != 0);
-          tc_mma(tm + 256 * o, umma_desc(Plo + s * 4096, 2048, 128), b, kIdO, 1);
+          tc_mma(tm + dcol, umma_desc(Phi + s * 4096, 2048, 128), b, os == 4 ? kIdO4 : kIdO, s != 0);
+          tc_mma(tm + dcol, umma_desc(Plo + s * 4096, 2048, 128), b, os == 4 ? kIdO4 : kIdO, 1);
         }
         tc_commit(&m->empty[g % kStages]);
       }
@@ -1313,8 +1316,8 @@ __device__ __forceinline__ void mla_consume(const KParams& P, const OpDesc& od, 
   mbar_wait(&m->mma_bar, (nmma + 1) & 1, P, &m->abort, op, t);
   __syncwarp();
   tc_fence_after();
-  // all 512 columns (256 per warp half), or this task's 256 (128 per warp half)
-  const int ncc = os > 1 ? 4 : 8, col0 = os > 1 ? 256 * part + 128 * half : 256 * half;
+  // this task's kvl / os columns, half of them per warp half, 32 per read
+  const int ncols = kvl / os, ncc = ncols / 64, col0 = ncols * part + (ncols / 2) * half;
   float* tile = reinterpret_cast<float*>(S.work) + warp * (32 * 36);  // [32 heads][36] (P is dead)
 #pragma unroll 1
   for (int cc = 0; cc < ncc; ++cc) {
@@ -1585,8 +1588,11 @@ __device__ void producer_loop(const KParams& P, const Smem& S) {
           __syncwarp();
         }
         for (int j = early; j < nS && ok; ++j) ok = issue(q + j * 16384, 16384, blk + j * 8192, 8192, 16384, pol_kv);
-        for (int o = 0; o < od.kvl / 256 && ok; ++o)
-          if (os == 1 || o == part) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
+        if (os == 4)  // a quarter of the columns: 16 contiguous 8-dim groups, 16 KB
+          ok = issue(blk + part * 16384, 16384, nullptr, 0, 0, pol_kv);
+        else
+          for (int o = 0; o < od.kvl / 256 && ok; ++o)
+            if (os == 1 || o == part) ok = issue(blk + o * 32768, 32768, nullptr, 0, 0, pol_kv);
       }
     }
   }
