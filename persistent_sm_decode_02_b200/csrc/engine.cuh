@@ -490,13 +490,49 @@ __device__ __forceinline__ void prologue(const OpDesc& od, int group, int task, 
       const int h0 = group, nh = 1;
       float* wt = reinterpret_cast<float*>(S.work + kCombineOff);  // [nh][nch]
       const int warp = tid >> 5;
+      const int hd = od.hdim;
+      // MLA blocks past position pos hold no partials
+      const int nc = min(od.nch, m->st.pos / kMlaBlock + 1);
+      if (n == 4 * kConsumers / 2 && hd == n) {
+        // One head of 512 columns: each half of the threads sums half of the blocks for its
+        // 4 columns (the first kB partial loads issued before the combine weights are known),
+        // and the two halves meet in shared memory.
+        constexpr int kB = 9;
+        const int hf = tid / (kConsumers / 2), e = 4 * (tid % (kConsumers / 2));
+        const int mid = (nc + 1) / 2, cb = hf ? mid : 0, ce = hf ? nc : mid;
+        const float* src = od.ao + (size_t)h0 * od.nch * hd + e;
+        float4 a[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) a[b] = cb + b < ce ? ldcg4(src + (size_t)(cb + b) * hd) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (warp == 0) combine_weights(od.am + (size_t)h0 * od.nch, od.al + (size_t)h0 * od.nch, od.nch, wt);
+        named_bar_sync(1, kConsumers);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = cb; c0 < ce; c0 += kB) {
+          if (c0 != cb)
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+              a[b] = c0 + b < ce ? ldcg4(src + (size_t)(c0 + b) * hd) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int b = 0; b < kB; ++b)
+            if (c0 + b < ce) fma4(acc, wt[c0 + b], a[b]);
+        }
+        float4* other = reinterpret_cast<float4*>(S.work + kCombineOff) + 64;  // behind the weights
+        if (hf) other[tid % (kConsumers / 2)] = acc;
+        named_bar_sync(1, kConsumers);
+        if (!hf) {
+          const float4 o2 = other[tid];
+          acc.x += o2.x;
+          acc.y += o2.y;
+          acc.z += o2.z;
+          acc.w += o2.w;
+          store_x4(x, bf, e, acc);
+        }
+        break;
+      }
       for (int h = warp; h < nh; h += kConsumerWarps)
         combine_weights(od.am + (size_t)(h0 + h) * od.nch, od.al + (size_t)(h0 + h) * od.nch, od.nch,
                         wt + h * od.nch);
       named_bar_sync(1, kConsumers);
-      const int hd = od.hdim;
-      // MLA blocks past position pos hold no partials
-      const int nc = min(od.nch, m->st.pos / kMlaBlock + 1);
       for (int e = 4 * tid; e < n; e += 4 * kConsumers) {
         const int h = e / hd, d = e % hd;
         const float* w = wt + h * od.nch;
