@@ -1,6 +1,7 @@
 /*
  * dec.h -- C ABI of a batch-1 transformer decode step run as one persistent
- * CUDA kernel per step on an NVIDIA B200 (sm_100a).
+ * CUDA kernel per step on an NVIDIA B200 (sm_100a), or a whole generation of
+ * many steps in one launch (dec_generate*).
  *
  * The problem statement follows the pages on TileRT (SemiAnalysis, "Ultra-High
  * Interactivity on NVIDIA GPUs? -- TileRT InferenceX", and "TileRT 是什么"):
@@ -9,8 +10,9 @@
  *   - a lifecycle of init / step / reset / cleanup (TileRT 是什么 §六 6.1: the
  *     prepare_money / show_hands / reset / go_home entry points);
  *   - the whole decode step as one persistent kernel whose tile tasks overlap
- *     weight streaming with compute (InferenceX article, "what TileRT is";
- *     TileRT 是什么 §二 2.2, tile-level runtime engine);
+ *     weight streaming with compute, launched once for a decode lifetime
+ *     (InferenceX article, "what TileRT is"; TileRT 是什么 §二 2.2, tile-level
+ *     runtime engine);
  *   - model structure: dense GQA, or MLA attention with a latent kv_cache and a
  *     RoPE-key pe_cache plus a routed MoE (TileRT 是什么 §五 5.2 and 5.3).
  *
