@@ -19,8 +19,12 @@ from synth import workloads
 
 pytestmark = pytest.mark.gpu
 
+# cases beyond the named workloads: name -> (workload, overrides).  The long-context MLA case has
+# 40 cache blocks, so the MLA attention runs two tasks per block (half of O's columns each); the
+# named small MLA case (2 blocks) runs four, and the full-size 8k workloads one.
+VARIANTS = {"small_mla_moe_fp8_ctx2500": ("small_mla_moe_fp8", dict(ctx=2500, cache_from="synthetic"))}
 SMALL = ["tiny_dense_f32", "small_dense_bf16", "small_dense_fp8", "small_dense_g8_bf16", "small_dense_g8_fp8_hd64",
-         "small_mla_moe_fp8"]
+         "small_mla_moe_fp8", "small_mla_moe_fp8_ctx2500"]
 MARGIN = 1e-4
 
 
@@ -41,7 +45,8 @@ _REF = {}
 def reference(name):
     """Oracle run of the workload: context, then n_decode teacher-forced steps."""
     if name not in _REF:
-        w = workloads.get(name)
+        base, over = VARIANTS.get(name, (name, {}))
+        w = workloads.get(base, **over)
         dec, first, _ = om.build_context(w)
         cache = dec.export_cache()
         steps, tok = [], first
