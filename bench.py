@@ -372,7 +372,9 @@ def main():
         line = {
             "impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": 0,
             "steps": r["steps"], "warmup": 1, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64 (bf16 rounding points of the model definition)", "data": "synthetic",
+            "dtype": "f64 (bf16 rounding points of the model definition)",
+            "data": "synthetic: seeded weights and seeded cache draw (an oracle step costs the same for any "
+                    "cache values, so this times the same work as a decoded context)",
             "config": {"workload": args.workload, "context": w["ctx"]},
             "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
                              "sample": f"{r['steps']} full oracle decode steps (all layers), host weight "
