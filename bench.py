@@ -4,14 +4,17 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 Prints one JSON line.  The default workload is the 12-layer MoE + MLA FP8 model
-with a 1k prefilled context (decode 1k), the shape the roofline target is set
-on.  Timing: W untimed warm-up steps, then K decode steps chained on the
+with a 1k context (decode 1k), the shape the roofline target is set on; the
+context is decoded on the GPU from its token ids before anything is timed
+(--cache synthetic installs the seeded cache draw instead).  Timing: W untimed
+warm-up steps, then K decode steps chained on the
 device (each step feeds back its own greedy token) between CUDA events on the
 decoder's stream; the step reads ~8 GB of weights, far more than the 126 MB L2,
 so no flush is needed.  `e2e` repeats the measurement through the synchronous
 C-ABI call dec_step with the token passed from the host and the greedy token
 read back every step.  `ablation` runs the same tiles as one kernel per op
-(plain launches and a CUDA graph).  `cpu_baseline` times the CPU oracle.
+(plain launches and a CUDA graph), and the K steps as one launch of a whole
+generation (dec_generate).  `cpu_baseline` times the CPU oracle.
 Under torchrun each rank runs an independent replica of the decoder on its own
 GPU (batch-1 decode does not shard here); value = all ranks' tokens / max time.
 """
