@@ -22,9 +22,12 @@ pytestmark = pytest.mark.gpu
 # cases beyond the named workloads: name -> (workload, overrides).  The long-context MLA case has
 # 40 cache blocks, so the MLA attention runs two tasks per block (half of O's columns each); the
 # named small MLA case (2 blocks) runs four, and the full-size 8k workloads one.
-VARIANTS = {"small_mla_moe_fp8_ctx2500": ("small_mla_moe_fp8", dict(ctx=2500, cache_from="synthetic"))}
+# The long-context dense case spreads 10,000 positions over 64 chunks per kv head, so each attention
+# task streams several ring stages and the last task of a kv head combines many chunks.
+VARIANTS = {"small_mla_moe_fp8_ctx2500": ("small_mla_moe_fp8", dict(ctx=2500, cache_from="synthetic")),
+            "small_dense_fp8_ctx10000": ("small_dense_fp8", dict(ctx=10000, cache_from="synthetic"))}
 SMALL = ["tiny_dense_f32", "small_dense_bf16", "small_dense_fp8", "small_dense_g8_bf16", "small_dense_g8_fp8_hd64",
-         "small_mla_moe_fp8", "small_mla_moe_fp8_ctx2500"]
+         "small_mla_moe_fp8", "small_mla_moe_fp8_ctx2500", "small_dense_fp8_ctx10000"]
 MARGIN = 1e-4
 
 
